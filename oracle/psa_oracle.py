@@ -1,0 +1,356 @@
+"""CPU oracle for the Pyramid Sparse Attention (PSA) forward pass, in float64.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or run
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+and reference legs of ``bench.py`` use it.  It shares no code with the CUDA
+path.
+
+Sources (the web pages describing PSA, arXiv:2512.04025):
+  [abs]  "PSA: Pyramid Sparse Attention for Efficient Video Understanding and
+         Generation" (chatpaper.ai), abstract: each query block gives every KV
+         block a pooling level, lower levels to critical blocks, higher levels
+         to less important ones, or prunes it; the kernel decouples the logical
+         block size from the hardware tile.
+  [news] top168.com article on arXiv:2512.04025: the pyramid's bottom level is
+         the original KV and every level above is average-pooled and coarser;
+         three components (pyramid KV blocks built by progressive pooling, a
+         multi-level mask generator driven by query-key block importance, and
+         adaptive pyramid attention that keeps the probability distribution
+         consistent); threshold-based assignment beats quantile-based.
+  [skill] "Psa Pyramid Sparse Attention" (skillmd.com), "Core Technique": levels
+         0/1/2/3 are the KV pooled 1x/2x/4x/8x.
+
+Where the pages leave a step open, the reading used is stated at the function.
+Every function below works on one (batch, head) slice; ``psa_forward`` loops.
+
+Notation: N tokens, d head dim, bq / bk query / KV block size, f_l = 2**l the
+pool factor of level l, s = softmax scale (1/sqrt(d) unless given).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Dict, Optional, Sequence, Tuple
+
+import numpy as np
+
+PRUNED = -1
+POOL = (1, 2, 4, 8)
+
+
+def cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+# --------------------------------------------------------------------- pyramid
+
+def pool_tokens(x: np.ndarray, f: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Average-pool tokens by factor f ([news] pyramid paragraph; [skill] Core
+    Technique, pooled KV cache).
+
+    Pooled token g is the mean of rows [g*f, min((g+1)*f, N)); the returned
+    counts c_g are the number of rows averaged (f except in a ragged tail).
+    x: [N, d] float64.  Returns ([ceil(N/f), d], [ceil(N/f)] int)."""
+    N, d = x.shape
+    G = cdiv(N, f)
+    full = N // f
+    out = np.empty((G, d), dtype=np.float64)
+    counts = np.full(G, f, dtype=np.int64)
+    out[:full] = x[:full * f].reshape(full, f, d).mean(axis=1)
+    if G > full:                                   # ragged tail group
+        out[full] = x[full * f:].mean(axis=0)
+        counts[full] = N - full * f
+    return out, counts
+
+
+@dataclass
+class Pyramid:
+    """Levels l = 0..3 of K and V of one head: keys[l], values[l] are
+    [ceil(N/f_l), d]; counts[l] the tokens behind each pooled row."""
+    keys: Dict[int, np.ndarray]
+    values: Dict[int, np.ndarray]
+    counts: Dict[int, np.ndarray]
+    N: int
+
+
+def build_pyramid(K: np.ndarray, V: np.ndarray, pool: Sequence[int] = POOL) -> Pyramid:
+    """Pyramid KV construction ([news] component one; [skill] levels 0..3).
+
+    Level 0 is K/V itself; level l pools the original tokens directly by f_l.
+    The article says the levels are built progressively; in exact arithmetic,
+    pooling level l-1 by 2 with count weights equals pooling level 0 by f_l, so
+    the oracle takes the direct form (a test checks the two agree)."""
+    N = K.shape[0]
+    keys, values, counts = {}, {}, {}
+    for l, f in enumerate(pool):
+        if f == 1:
+            keys[l], values[l] = K.astype(np.float64), V.astype(np.float64)
+            counts[l] = np.ones(N, dtype=np.int64)
+        else:
+            keys[l], counts[l] = pool_tokens(K, f)
+            values[l], _ = pool_tokens(V, f)
+    return Pyramid(keys, values, counts, N)
+
+
+def block_rows(j: int, l: int, bk: int, pyr: Pyramid, pool: Sequence[int] = POOL) -> range:
+    """Rows of level l that summarise KV block j: [j*bk/f_l, min((j+1)*bk/f_l, rows_l))."""
+    f = pool[l]
+    per = bk // f
+    return range(j * per, min((j + 1) * per, pyr.keys[l].shape[0]))
+
+
+# ------------------------------------------------------------ mask generation
+
+def query_block_means(Q: np.ndarray, bq: int) -> np.ndarray:
+    """q_bar[a] = mean of the valid rows of query block a.  The pages score
+    query-key block pairs ([news] component two) without saying how a query
+    block is summarised; the mean is the reading used.  Returns [Nq, d]."""
+    N = Q.shape[0]
+    Nq = cdiv(N, bq)
+    return np.stack([Q[a * bq:min((a + 1) * bq, N)].mean(axis=0) for a in range(Nq)])
+
+
+def block_logits(qbar: np.ndarray, pyr: Pyramid, bk: int, scale: float,
+                 pool: Sequence[int] = POOL) -> np.ndarray:
+    """Block importance z[a, j] ([news] component two; [skill] block scoring).
+
+    Reading: the query-block mean is scored against the coarsest (level-3)
+    pooled keys of block j, and the block's logit is the log of the softmax mass
+    those pooled keys stand for: z = logsumexp_g(s * q_bar . K3[g] + ln c_g).
+    For a block whose tokens are identical this is exactly the logsumexp of the
+    block's own token logits.  Returns [Nq, Nk]."""
+    L = len(pool) - 1
+    K3, c3 = pyr.keys[L], pyr.counts[L]
+    Nq, Nk = qbar.shape[0], cdiv(pyr.N, bk)
+    z = np.empty((Nq, Nk), dtype=np.float64)
+    logits = scale * (qbar @ K3.T) + np.log(c3)[None, :]
+    for j in range(Nk):
+        rows = block_rows(j, L, bk, pyr, pool)
+        part = logits[:, rows.start:rows.stop]
+        m = part.max(axis=1, keepdims=True)
+        z[:, j] = m[:, 0] + np.log(np.exp(part - m).sum(axis=1))
+    return z
+
+
+def visible(a: int, j: int, N: int, bq: int, bk: int, causal: bool) -> bool:
+    """Causal: KV block j is visible to query block a iff its first token is at
+    or before the query block's last row."""
+    if not causal:
+        return True
+    return j * bk <= min((a + 1) * bq, N) - 1
+
+
+def straddles(a: int, j: int, N: int, bq: int, bk: int) -> bool:
+    """Causal: KV block j overlaps the row range of query block a, so a token
+    mask (key position <= query position) is needed inside it."""
+    q_lo, q_hi = a * bq, min((a + 1) * bq, N) - 1
+    k_lo, k_hi = j * bk, min((j + 1) * bk, N) - 1
+    return k_lo <= q_hi and k_hi >= q_lo
+
+
+@dataclass
+class MaskResult:
+    level_map: np.ndarray    # int8 [Nq, Nk]; -1 = pruned
+    mass: np.ndarray         # P[a, j], softmax over visible blocks (0 for invisible)
+    cum_before: np.ndarray   # C[a, j]: mass of the blocks ranked before j in row a
+    rank: np.ndarray         # rank of j in row a (visible blocks only; -1 otherwise)
+
+
+def rank_blocks(z_row: np.ndarray, vis: np.ndarray):
+    """One query block's softmax over its visible KV blocks, ranked.
+
+    P = softmax(z) over the visible blocks ``vis``; the ranking is P descending
+    with ties going to the lower block index; C[r] is the mass of the blocks
+    ranked before r (exclusive prefix, summed in rank order).
+    Returns (order: block indices by rank, P in rank order, C in rank order)."""
+    zz = z_row[vis]
+    p = np.exp(zz - zz.max())
+    p = p / p.sum()
+    idx = np.lexsort((vis, -p))            # primary key -P, then block index
+    p_sorted = p[idx]
+    c = np.concatenate(([0.0], np.cumsum(p_sorted)[:-1]))
+    return vis[idx], p_sorted, c
+
+
+def level_of(c: np.ndarray, tau: Sequence[float]) -> np.ndarray:
+    """level = the smallest l with C < tau_l, else pruned (-1)."""
+    out = np.full(c.shape, PRUNED, dtype=np.int8)
+    for l in reversed(range(len(tau))):
+        out[c < tau[l]] = l
+    return out
+
+
+def apply_overrides(row: np.ndarray, a: int, N: int, bq: int, bk: int, causal: bool,
+                    forced_prefix_tokens: int) -> None:
+    """In place: causal blocks after the query block are pruned and blocks
+    straddling its diagonal get level 0; visible blocks holding any of the first
+    ``forced_prefix_tokens`` tokens get level 0."""
+    j = np.arange(row.shape[0])
+    q_lo, q_hi = a * bq, min((a + 1) * bq, N) - 1
+    vis = (j * bk <= q_hi) if causal else np.ones(row.shape[0], dtype=bool)
+    strad = vis & (np.minimum((j + 1) * bk, N) - 1 >= q_lo) if causal else ~vis
+    forced = vis & (j * bk < forced_prefix_tokens)
+    row[~vis] = PRUNED
+    row[strad | forced] = 0
+
+
+def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
+                  causal: bool = False, forced_prefix_tokens: int = 0) -> MaskResult:
+    """Threshold-based multi-level mask ([news] ablations: threshold-based
+    assignment; [abs] lower levels to critical blocks, higher to less important).
+
+    For each query block a: P = softmax over visible j of z[a, j]; rank blocks by
+    P descending, ties to the lower j; C_r = mass of the blocks ranked before r;
+    level = the smallest l with C_r < tau_l, else pruned.  Then the overrides of
+    ``apply_overrides``.  Readings: the exclusive cumulative mass (so the top
+    block always gets level 0) and the override order are this build's."""
+    Nq, Nk = z.shape
+    level_map = np.full((Nq, Nk), PRUNED, dtype=np.int8)
+    mass = np.zeros((Nq, Nk), dtype=np.float64)
+    cum = np.zeros((Nq, Nk), dtype=np.float64)
+    rank = np.full((Nq, Nk), -1, dtype=np.int64)
+    for a in range(Nq):
+        vis = np.array([j for j in range(Nk) if visible(a, j, N, bq, bk, causal)])
+        order, p, c = rank_blocks(z[a], vis)
+        mass[a, order], cum[a, order] = p, c
+        rank[a, order] = np.arange(len(order))
+        level_map[a, order] = level_of(c, tau)
+        apply_overrides(level_map[a], a, N, bq, bk, causal, forced_prefix_tokens)
+    return MaskResult(level_map, mass, cum, rank)
+
+
+# ----------------------------------------------------------------- attention
+
+def pyramid_attention(Q: np.ndarray, pyr: Pyramid, level_map: np.ndarray, bq: int, bk: int,
+                      scale: float, causal: bool = False,
+                      pool: Sequence[int] = POOL) -> Tuple[np.ndarray, np.ndarray]:
+    """Adaptive pyramid attention ([news] component three, keeping the
+    probability distribution consistent).
+
+    Row i of query block a takes ONE softmax over every key it keeps: for each
+    block j with level l = map[a, j] >= 0, the level-l pooled rows of block j,
+    each with logit s * q_i . K_l[g] + ln c_g.  The ln c_g term lets a pooled key
+    carry the softmax mass of the c_g tokens it averages: it equals attending to
+    the pooled key repeated c_g times.  Causal blocks straddling the diagonal
+    (always level 0) also mask keys after row i.  A row that keeps no key gets
+    O = 0 and LSE = -inf.  Returns (O [N, d], LSE [N], natural log)."""
+    N, d = Q.shape
+    Nq, Nk = level_map.shape
+    O = np.zeros((N, d), dtype=np.float64)
+    lse = np.full(N, -np.inf, dtype=np.float64)
+    for a in range(Nq):
+        ks, vs, bias, kpos = [], [], [], []
+        for j in range(Nk):
+            l = int(level_map[a, j])
+            if l < 0:
+                continue
+            rows = block_rows(j, l, bk, pyr, pool)
+            ks.append(pyr.keys[l][rows.start:rows.stop])
+            vs.append(pyr.values[l][rows.start:rows.stop])
+            bias.append(np.log(pyr.counts[l][rows.start:rows.stop]))
+            # token position of each key; pooled keys (level > 0) never straddle.
+            kpos.append(np.arange(rows.start, rows.stop) * pool[l] if l == 0
+                        else np.full(len(rows), -1))
+        if not ks:
+            continue
+        Kk, Vk = np.concatenate(ks), np.concatenate(vs)
+        bias_a, kpos_a = np.concatenate(bias), np.concatenate(kpos)
+        rows_i = np.arange(a * bq, min((a + 1) * bq, N))
+        # every row of block a keeps the same keys: one matrix product per block
+        logit = scale * (Q[rows_i] @ Kk.T) + bias_a[None, :]
+        if causal:
+            logit = np.where(kpos_a[None, :] > rows_i[:, None], -np.inf, logit)
+        m = logit.max(axis=1)
+        ok = np.isfinite(m)
+        w = np.exp(logit[ok] - m[ok, None])
+        ssum = w.sum(axis=1)
+        O[rows_i[ok]] = (w @ Vk) / ssum[:, None]
+        lse[rows_i[ok]] = m[ok] + np.log(ssum)
+    return O, lse
+
+
+# ------------------------------------------------------------------- driver
+
+@dataclass
+class HeadResult:
+    O: np.ndarray
+    lse: np.ndarray
+    mask: MaskResult
+    z: np.ndarray
+
+
+def psa_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, bq: int, bk: int,
+             tau: Sequence[float], causal: bool = False, forced_prefix_tokens: int = 0,
+             scale: Optional[float] = None, level_map: Optional[np.ndarray] = None,
+             pool: Sequence[int] = POOL) -> HeadResult:
+    """The whole PSA forward for one (batch, query head): pyramid, query-block
+    means, block logits, level assignment (unless ``level_map`` is given), then
+    pyramid attention.  Q [N, d]; K, V [N, d] of the matching KV head."""
+    N, d = Q.shape
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    pyr = build_pyramid(K, V, pool)
+    z = block_logits(query_block_means(Q, bq), pyr, bk, s, pool)
+    mask = assign_levels(z, tau, N, bq, bk, causal, forced_prefix_tokens)
+    lm = mask.level_map if level_map is None else level_map
+    O, lse = pyramid_attention(Q, pyr, lm, bq, bk, s, causal, pool)
+    return HeadResult(O, lse, mask, z)
+
+
+def executed_flops(level_map: np.ndarray, N: int, d: int, bq: int, bk: int,
+                   causal: bool = False, pool: Sequence[int] = POOL) -> float:
+    """FLOPs the method executes for one head's map: 4*d per (query row, kept
+    key); a causal block straddling the diagonal counts only unmasked pairs."""
+    Nq, Nk = level_map.shape
+    qrows = np.array([min((a + 1) * bq, N) - a * bq for a in range(Nq)], dtype=np.float64)
+    valid = np.array([min((j + 1) * bk, N) - j * bk for j in range(Nk)], dtype=np.int64)
+    keys = np.zeros((Nk, len(pool) + 1), dtype=np.float64)   # column -1 <- pruned = 0
+    for l, f in enumerate(pool):
+        keys[:, l] = -(-valid // f)
+    per = keys[np.arange(Nk)[None, :], level_map.astype(np.int64)]   # [Nq, Nk]
+    total = float((qrows[:, None] * per).sum())
+    if causal:
+        for a in range(Nq):
+            i = np.arange(a * bq, min((a + 1) * bq, N))
+            for j in range(Nk):
+                if level_map[a, j] >= 0 and straddles(a, j, N, bq, bk):
+                    k_lo, k_hi = j * bk, min((j + 1) * bk, N)
+                    exact = np.maximum(0, np.minimum(k_hi, i + 1) - k_lo).sum()
+                    total += float(exact) - qrows[a] * per[a, j]
+    return 4.0 * d * total
+
+
+@dataclass
+class ForwardResult:
+    O: np.ndarray            # [B, Hq, N, d]
+    lse: np.ndarray          # [B, Hq, N]
+    level_map: np.ndarray    # int8 [B, Hq, Nq, Nk]
+    mass: np.ndarray         # [B, Hq, Nq, Nk]
+    cum_before: np.ndarray   # [B, Hq, Nq, Nk]
+
+
+def psa_forward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, bq: int, bk: int,
+                tau: Sequence[float], causal: bool = False, forced_prefix_tokens: int = 0,
+                scale: Optional[float] = None, level_map: Optional[np.ndarray] = None,
+                heads: Optional[Sequence[Tuple[int, int]]] = None) -> ForwardResult:
+    """PSA forward over [B, Hq, N, d] queries and [B, Hkv, N, d] keys/values
+    (float64).  Query head h reads KV head h // (Hq / Hkv) (grouped queries);
+    maps are per query head.  ``heads`` restricts the work to some (b, h) pairs
+    (the others stay zero / pruned)."""
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    grp = Hq // Hkv
+    Nq, Nk = cdiv(N, bq), cdiv(N, bk)
+    O = np.zeros_like(Q, dtype=np.float64)
+    lse = np.full((B, Hq, N), -np.inf)
+    lm = np.full((B, Hq, Nq, Nk), PRUNED, dtype=np.int8)
+    mass = np.zeros((B, Hq, Nq, Nk))
+    cum = np.zeros((B, Hq, Nq, Nk))
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in todo:
+        r = psa_head(Q[b, h], K[b, h // grp], V[b, h // grp], bq, bk, tau, causal,
+                     forced_prefix_tokens, scale,
+                     None if level_map is None else level_map[b, h])
+        O[b, h], lse[b, h] = r.O, r.lse
+        lm[b, h] = r.mask.level_map if level_map is None else level_map[b, h]
+        mass[b, h], cum[b, h] = r.mask.mass, r.mask.cum_before
+    return ForwardResult(O, lse, lm, mass, cum)

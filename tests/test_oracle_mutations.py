@@ -1,0 +1,79 @@
+"""Planted mistakes: each mutation below breaks one step of a copy of the
+oracle (the source text is edited and loaded as a fresh module, on the CPU), and
+at least one pin must then fail.  This shows the pins are tight enough to catch
+a dropped term, a wrong sign or index, or a swapped operand."""
+import os
+import sys
+import types
+
+import numpy as np
+import pytest
+
+from tests import oracle_pins as P
+from tests.bruteforce import psa_bruteforce
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "psa_oracle.py")
+
+MUTATIONS = {
+    "attention drops ln c": ("+ bias_a[None, :]", ""),
+    "attention forgets the scale": ("scale * (Q[rows_i] @ Kk.T)", "(Q[rows_i] @ Kk.T)"),
+    "causal mask off by one": ("kpos_a[None, :] > rows_i[:, None]", "kpos_a[None, :] >= rows_i[:, None]"),
+    "inclusive cumulative mass": ("np.concatenate(([0.0], np.cumsum(p_sorted)[:-1]))", "np.cumsum(p_sorted)"),
+    "ties to the higher index": ("np.lexsort((vis, -p))", "np.lexsort((-vis, -p))"),
+    "ascending rank": ("np.lexsort((vis, -p))", "np.lexsort((vis, p))"),
+    "threshold <= instead of <": ("out[c < tau[l]] = l", "out[c <= tau[l]] = l"),
+    "block logit drops ln c": ("+ np.log(c3)[None, :]", ""),
+    "block logit uses level 2": ("L = len(pool) - 1", "L = len(pool) - 2"),
+    "pool drops the tail": ("out[full] = x[full * f:].mean(axis=0)", "out[full] = x[full * f - 1:].mean(axis=0)"),
+    "pool counts wrong": ("counts[full] = N - full * f", "counts[full] = f"),
+    "query mean includes next block": ("Q[a * bq:min((a + 1) * bq, N)].mean(axis=0)", "Q[a * bq:min((a + 1) * bq + 1, N)].mean(axis=0)"),
+    "straddle test shifted": ("np.minimum((j + 1) * bk, N) - 1 >= q_lo", "np.minimum((j + 1) * bk, N) - 1 > q_lo + 63"),
+    "forced prefix ignored": ("row[strad | forced] = 0", "row[strad] = 0"),
+    "values pooled from keys": ("values[l], _ = pool_tokens(V, f)", "values[l], _ = pool_tokens(K, f)"),
+}
+
+
+def _mutant(old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, old
+    name = "oracle_mutant_%d" % abs(hash((old, new)))
+    mod = types.ModuleType(name)
+    sys.modules[name] = mod            # dataclasses look their module up
+    try:
+        exec(compile(src.replace(old, new), name, "exec"), mod.__dict__)
+    finally:
+        sys.modules.pop(name, None)
+    return mod
+
+
+def _bruteforce_agrees(M):
+    rng = np.random.default_rng(21)
+    for N, d, bq, causal, forced in ((203, 8, 64, False, 70), (187, 4, 64, True, 0),
+                                     (509, 8, 64, False, 0)):
+        Q, K, V = (rng.standard_normal((N, d)) * 1.5 for _ in range(3))
+        tau = (0.5, 0.7, 0.85, 0.95)
+        O_b, _, lv = psa_bruteforce(Q.tolist(), K.tolist(), V.tolist(), bq, 64, tau, causal, forced)
+        r = M.psa_head(Q, K, V, bq, 64, tau, causal, forced)
+        if r.mask.level_map.tolist() != lv or not np.allclose(r.O, np.array(O_b), atol=1e-10):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught_by_a_pin(name):
+    M = _mutant(*MUTATIONS[name])
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(M)
+        except Exception:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches mutation '{name}'"
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught_by_bruteforce(name):
+    if name in ("threshold <= instead of <", "ties to the higher index"):
+        pytest.skip("random masses never tie or land on a threshold; the golden cases pin these")
+    assert not _bruteforce_agrees(_mutant(*MUTATIONS[name]))
