@@ -1,0 +1,320 @@
+"""Benchmark of the PSA forward pass (pyramid -> mask -> attention) on B200.
+
+One step = one whole forward pass over one batch of the workload (default: the
+Wan2.1-1.3B-shaped video DiT self-attention, B=1, H=12, N=32760, d=128, bf16,
+128/64 blocks, thresholds frozen for 91% skipped dense FLOPs).  Inputs are the
+seeded synthetic smooth-field-plus-noise tensors of ``workloads``.
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+batch (independent problems, no data-path collective: weak scaling); the
+timing is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "PSA fwd ms/call & dense-equiv TFLOP/s at Wan-1.3B shape; % bf16 tensor peak"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="wan2.1_1.3b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-heads", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- CPU oracle leg
+
+def cpu_sample(w: W.Workload, n_heads: int):
+    """Time the oracle (as it stands) on `n_heads` whole heads of the workload.
+    Returns (dense-equivalent TFLOP/s, seconds, cores, sample description)."""
+    import oracle as O
+    cores = len(os.sched_getaffinity(0))
+    grp = w.Hq // w.Hkv
+    heads = list(range(n_heads))
+    inp = W.make_inputs(w, heads_q=heads, heads_kv=sorted({h // grp for h in heads}))
+    tau = W.thresholds(w)
+    t0 = time.perf_counter()
+    for h in heads:
+        O.psa_head(inp.as_f64("q", 0, h), inp.as_f64("k", 0, h // grp), inp.as_f64("v", 0, h // grp),
+                   w.q_blk, w.kv_blk, tau, w.causal, w.forced_prefix_tokens)
+    dt = time.perf_counter() - t0
+    dense = w.dense_flops() / (w.B * w.Hq) * n_heads
+    return (dense / dt / 1e12, dt, cores,
+            f"{n_heads} of {w.B * w.Hq} heads of {w.name}, whole forward (pyramid, mask, attention), "
+            f"NumPy float64, BLAS threads = {cores}")
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = W.BY_NAME[args.workload]
+    times, val = [], None
+    for _ in range(args.warmup):
+        cpu_sample(w, 1)
+    for _ in range(args.steps):
+        val, dt, cores, sample = cpu_sample(w, 1)
+        times.append(dt)
+    tot = sum(times)
+    dense_head = w.dense_flops() / (w.B * w.Hq)
+    value = dense_head * len(times) / tot / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "sample": "one head per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------- clock sampler
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _loop(self):
+        nv = self.nv
+        names = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                 "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4, "sync_boost": 0x10}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._loop, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------- our leg
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import level_sparse_attention_b200 as P
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.BY_NAME[args.workload]
+    tau = W.thresholds(w)
+    p = P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk, tau, w.causal,
+                      w.forced_prefix_tokens, 0.0,
+                      torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+    inp = W.make_inputs(w)
+
+    def host(x):
+        t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
+            else torch.from_numpy(x)
+        return t.pin_memory()
+
+    hq, hk, hv = host(inp.q), host(inp.k), host(inp.v)
+    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    ws = P.new_workspace(p, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lm = torch.empty(P.map_shape(p), dtype=torch.int8, device=dev)
+
+    def step():
+        P.build_pyramid(p, k, v, ws)
+        P.score_and_mask(p, q, ws, lm)
+        P.attention_fwd(p, q, k, v, ws, out, lse)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    P.check_device(p, ws)
+
+    # executed (algorithmic) attention FLOPs of this map: 4*d*sum(valid q rows * kept keys)
+    counts = P.workspace_view(ws, P.workspace_layout(p)["counts"], (w.B, w.Hq, w.Nq, 4),
+                              torch.int32).cpu().numpy().astype(np.int64)
+    keys_per_row = counts[..., 0] * 64 + counts[..., 1] * 32 + counts[..., 2] * 16 + counts[..., 3] * 8
+    qrows = np.array([min(w.q_blk, w.N - a * w.q_blk) for a in range(w.Nq)], dtype=np.int64)
+    executed = float(4 * w.d * (keys_per_row * qrows[None, None, :]).sum())
+    # (tail KV blocks and the causal diagonal make this an upper bound of a few
+    #  keys per row; the oracle's executed_flops is exact)
+    dense = w.dense_flops()
+    padded_keys = float(np.ceil(keys_per_row / 128.0).sum() * 128)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()                       # L2 flush outside the timed events
+            e = ev[i]
+            e[0].record(stream)
+            P.build_pyramid(p, k, v, ws)
+            e[1].record(stream)
+            P.score_and_mask(p, q, ws, lm)
+            e[2].record(stream)
+            P.attention_fwd(p, q, k, v, ws, out, lse)
+            e[3].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    pyr_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    mask_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    tot_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms = tot_ms / args.steps
+    value = dense * world / (ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D of Q, K, V, the
+    # forward, D2H of O, every step inside the timed region
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        P.forward(p, q, k, v, out, ws, lse)
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    P.check_device(p, ws)
+
+    bf16_peak, hbm_peak, peak_kind = peaks()
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    achieved = executed / (attn_avg * 1e-3) / 1e12
+    es = 2 if w.dtype == "bf16" else 4
+    pyr_bytes = 2 * w.B * w.Hkv * w.N * w.d * es * (1 + 0.875) + w.B * w.Hkv * (-(-w.N // 8)) * w.d * 4
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        val, dt, cores, sample = cpu_sample(w, args.cpu_sample_heads)
+        cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(dt, 2)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded smooth 3-D field + noise)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "q_blk": w.q_blk, "kv_blk": w.kv_blk, "tau": [round(t, 6) for t in tau],
+                   "causal": w.causal, "skipped_dense_fraction": 1.0 - executed / dense,
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "parallelism": f"independent batch per GPU x{world}"},
+        "ms_per_call": ms, "pct_bf16_peak_dense_equiv": 100.0 * value / world / bf16_peak,
+        "executed_tflops": executed * world / (ms * 1e-3) / 1e12,
+        "kernel_ms": {"pyramid": sum(pyr_ms) / len(pyr_ms), "mask": sum(mask_ms) / len(mask_ms),
+                      "attention": attn_avg},
+        "pyramid_gbs": pyr_bytes / (sum(pyr_ms) / len(pyr_ms) * 1e-3) / 1e9,
+        "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": bf16_peak, "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s",
+                     "frac": achieved / bf16_peak, "traffic": None,
+                     "executed_flops_per_launch": executed,
+                     "padding_fraction": 1.0 - (keys_per_row.sum() / max(padded_keys, 1.0))},
+        "cpu_baseline": cpu,
+        "e2e": {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * es),
+                "d2h_bytes_per_step": int(out.numel() * es)},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,148 @@
+/*
+ * psa.h — C ABI of the B200 (sm_100a) Pyramid Sparse Attention forward pass.
+ *
+ * The method (arXiv:2512.04025, "PSA: Pyramid Sparse Attention for Efficient
+ * Video Understanding and Generation", abstract): instead of keeping or
+ * dropping whole KV blocks, each query block gives every KV block a pooling
+ * level — the KV block itself (level 0) or its 2x / 4x / 8x average-pooled
+ * form (levels 1..3) — or prunes it, and attends to the mixed-resolution keys
+ * with one softmax.  The top168.com article on the paper names the three
+ * components implemented here: pyramid KV construction by average pooling, a
+ * multi-level mask generator driven by query-key block importance with
+ * thresholds, and adaptive pyramid attention that keeps the probability
+ * distribution consistent (here: each pooled key's logit gets + ln(c), c the
+ * number of tokens it averages).
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    the library never allocates, frees or synchronises (psa_check_device is
+ *    the one call that waits on the stream).  All work is enqueued on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Tensors are dense row-major: Q/O [B, Hq, N, d], K/V [B, Hkv, N, d] with d
+ *    contiguous; element type is params->dtype (fp32 or bf16).  Device
+ *    pointers must be 16-byte aligned.
+ *  - Arguments are validated on the host before anything is launched; on an
+ *    error nothing is enqueued and a psa_status_t other than PSA_OK returns.
+ *    A CUDA launch error is returned as PSA_ERR_CUDA.
+ *  - Kernels never trap: a device wait that runs past its time limit sets an
+ *    error word in the workspace and the kernel returns early; read it with
+ *    psa_check_device (PSA_ERR_DEVICE_TIMEOUT).
+ */
+#ifndef PSA_H_
+#define PSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PSA_OK = 0,
+  PSA_ERR_INVALID_ARG = 1,          /* NULL pointer, bad size, tau not monotone, ... */
+  PSA_ERR_UNSUPPORTED = 2,          /* valid but not implemented (e.g. d = 96)        */
+  PSA_ERR_MISALIGNED = 3,           /* a device pointer is not 16-byte aligned         */
+  PSA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < psa_workspace_size(params)    */
+  PSA_ERR_CUDA = 5,                 /* a CUDA call or launch failed                    */
+  PSA_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up waiting (see psa_check_device) */
+} psa_status_t;
+
+typedef enum { PSA_F32 = 0, PSA_BF16 = 1 } psa_dtype_t;
+
+/* Problem description, shared by every entry point.
+ *  B, Hq, Hkv, N, d  batch, query heads, KV heads (Hq % Hkv == 0; query head h
+ *                    reads KV head h / (Hq / Hkv)), tokens, head dim (64 or 128).
+ *  q_blk, kv_blk     query block (64 or 128) and KV block (64) sizes, in tokens.
+ *  n_levels, pool    must be 4 and {1, 2, 4, 8}: level l pools 2^l tokens
+ *                    ("Psa Pyramid Sparse Attention", Core Technique).
+ *  tau               cumulative-mass thresholds, non-decreasing, in (0, 1]:
+ *                    a KV block ranked r gets the smallest level l with
+ *                    C_r < tau[l] (C_r = mass of the blocks ranked before it),
+ *                    else it is pruned.
+ *  causal            1: key position <= query position (blocks after the query
+ *                    block are pruned, blocks straddling its diagonal get level
+ *                    0 and a token mask).
+ *  forced_prefix_tokens  visible KV blocks holding any of the first this-many
+ *                    tokens get level 0 (e.g. a text prefix).
+ *  scale             softmax scale; 0 means 1/sqrt(d).
+ *  dtype             element type of Q, K, V, O and of the pooled levels.    */
+typedef struct {
+  int B, Hq, Hkv, N, d;
+  int q_blk, kv_blk;
+  int n_levels;
+  int pool[4];
+  float tau[4];
+  int causal;
+  int forced_prefix_tokens;
+  float scale;
+  psa_dtype_t dtype;
+} psa_params_t;
+
+/* Bytes of device workspace the calls below need for `params` (0 if params are
+ * invalid).  The workspace holds: a device error word; pooled K/V levels 1..3
+ * [B, Hkv, ceil(N/2^l), d] in dtype; level-3 keys in fp32 for scoring;
+ * query-block means; block logits; an internal level map; and the per-query-
+ * block work list (KV block indices sorted by level, then index).  It is owned
+ * by the caller and may be reused across calls with the same params. */
+size_t psa_workspace_size(const psa_params_t* params);
+
+/* Pyramid KV construction (top168.com article on PSA, pyramid paragraph and
+ * component one: bottom level = original KV, each level up average-pooled).
+ * K, V: device [B, Hkv, N, d].  Writes levels 1..3 of K and V and the fp32
+ * level-3 keys into `workspace`.  Pooled row g of level l is the mean of tokens
+ * [g*2^l, min((g+1)*2^l, N)), summed in fp32 and rounded once to dtype. */
+psa_status_t psa_build_pyramid(const psa_params_t* params, const void* K, const void* V,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Multi-level mask generation (top168.com article, component two and the
+ * threshold ablation; abstract of the paper: lower pooling levels for critical
+ * KV blocks).  Needs the pyramid from psa_build_pyramid in `workspace`.
+ * Q: device [B, Hq, N, d].  For each query block: q_bar = mean of its valid
+ * rows (fp32); block logit z_j = logsumexp over block j's level-3 keys g of
+ * (scale * q_bar . K3[g] + ln c_g); P = softmax over the visible blocks; rank
+ * by P descending (ties to the lower j); level from tau as in psa_params_t;
+ * then causal and forced-prefix overrides.  Writes the work list into
+ * `workspace` and, if non-NULL:
+ *   level_map  device int8 [B, Hq, ceil(N/q_blk), ceil(N/kv_blk)], -1 = pruned;
+ *   block_mass device fp32, same shape: P (0 for blocks after a causal query block). */
+psa_status_t psa_score_and_mask(const psa_params_t* params, const void* Q, void* workspace,
+                                size_t workspace_bytes, int8_t* level_map, float* block_mass,
+                                void* stream);
+
+/* Adaptive pyramid attention (top168.com article, component three; the
+ * paper's abstract: a kernel whose logical block size is decoupled from the
+ * hardware tile).  Row i of query block a takes one softmax over every kept
+ * key: for block j at level l = map[a][j] >= 0, block j's level-l pooled rows,
+ * logit scale * q_i . K_l[g] + ln c_g.  Q, K, V: device, as above; K and V are
+ * level 0 (the pyramid's other levels come from `workspace`).  level_map:
+ * device int8 map to use instead of the one psa_score_and_mask built (NULL =
+ * use the workspace's work list); a non-NULL map is turned into a work list
+ * in `workspace` first.  O: device [B, Hq, N, d] in dtype.  lse: device fp32
+ * [B, Hq, N] natural-log sum of exp of the logits, or NULL.  A row that keeps
+ * no key gets O = 0 and lse = -inf. */
+psa_status_t psa_attention_fwd(const psa_params_t* params, const void* Q, const void* K,
+                               const void* V, void* workspace, size_t workspace_bytes,
+                               const int8_t* level_map, void* O, float* lse, void* stream);
+
+/* The whole forward pass: psa_build_pyramid, psa_score_and_mask and
+ * psa_attention_fwd in that order on one stream.  level_map (optional output,
+ * device int8) receives the map that was used. */
+psa_status_t psa_forward(const psa_params_t* params, const void* Q, const void* K, const void* V,
+                         void* O, float* lse, int8_t* level_map, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Waits for `stream`, then reads and clears the workspace's device error word.
+ * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
+ * check, PSA_ERR_CUDA if the stream reported an error, else PSA_OK. */
+psa_status_t psa_check_device(const psa_params_t* params, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* psa_status_string(psa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PSA_H_ */

@@ -1,0 +1,201 @@
+"""Python binding of libpsa.so, the B200 (sm_100a) Pyramid Sparse Attention
+forward pass.  Argument marshalling only: every step runs in the library's CUDA
+kernels; torch supplies device memory and the current stream.
+
+The entry points mirror include/psa.h one to one (build_pyramid,
+score_and_mask, attention_fwd, forward, workspace_size, check_device); the
+helper ``psa_forward`` allocates the outputs and the workspace with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpsa.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "misaligned",
+           4: "workspace too small", 5: "CUDA error", 6: "device timeout"}
+
+
+class PSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Params(ctypes.Structure):
+    """Mirror of psa_params_t."""
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("N", ctypes.c_int), ("d", ctypes.c_int), ("q_blk", ctypes.c_int),
+                ("kv_blk", ctypes.c_int), ("n_levels", ctypes.c_int),
+                ("pool", ctypes.c_int * 4), ("tau", ctypes.c_float * 4),
+                ("causal", ctypes.c_int), ("forced_prefix_tokens", ctypes.c_int),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpsa.so (built by ``python -m level_sparse_attention_b200.build``).
+    There is no fallback: a missing library is an error."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; run python -m level_sparse_attention_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, vp, sz = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_size_t
+        sigs = {
+            "psa_workspace_size": (sz, [P]),
+            "psa_build_pyramid": (ctypes.c_int, [P, vp, vp, vp, sz, vp]),
+            "psa_score_and_mask": (ctypes.c_int, [P, vp, vp, sz, vp, vp, vp]),
+            "psa_attention_fwd": (ctypes.c_int, [P, vp, vp, vp, vp, sz, vp, vp, vp, vp]),
+            "psa_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "psa_check_device": (ctypes.c_int, [P, vp, sz, vp]),
+            "psa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
+            "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string")
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().psa_status_string(status).decode()
+    except ImportError:
+        return _STATUS.get(status, "unknown")
+
+
+def make_params(B: int, Hq: int, Hkv: int, N: int, d: int, q_blk: int = 128, kv_blk: int = 64,
+                tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97), causal: bool = False,
+                forced_prefix_tokens: int = 0, scale: float = 0.0,
+                dtype: torch.dtype = torch.bfloat16) -> Params:
+    p = Params()
+    p.B, p.Hq, p.Hkv, p.N, p.d = B, Hq, Hkv, N, d
+    p.q_blk, p.kv_blk, p.n_levels = q_blk, kv_blk, 4
+    for i in range(4):
+        p.pool[i] = 1 << i
+        p.tau[i] = float(tau[i])
+    p.causal, p.forced_prefix_tokens, p.scale = int(bool(causal)), forced_prefix_tokens, scale
+    p.dtype = BF16 if dtype == torch.bfloat16 else F32
+    return p
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise PSAError(status, where)
+
+
+def workspace_size(p: Params) -> int:
+    return int(lib().psa_workspace_size(ctypes.byref(p)))
+
+
+def new_workspace(p: Params, device="cuda") -> torch.Tensor:
+    n = workspace_size(p)
+    if n == 0:
+        raise PSAError(1, "psa_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def build_pyramid(p: Params, K: torch.Tensor, V: torch.Tensor, ws: torch.Tensor, stream=None):
+    _check(lib().psa_build_pyramid(ctypes.byref(p), _ptr(K), _ptr(V), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "psa_build_pyramid")
+
+
+def score_and_mask(p: Params, Q: torch.Tensor, ws: torch.Tensor,
+                   level_map: Optional[torch.Tensor] = None,
+                   block_mass: Optional[torch.Tensor] = None, stream=None):
+    _check(lib().psa_score_and_mask(ctypes.byref(p), _ptr(Q), _ptr(ws), ws.numel(),
+                                    _ptr(level_map), _ptr(block_mass), _stream(stream)),
+           "psa_score_and_mask")
+
+
+def attention_fwd(p: Params, Q, K, V, ws, O, lse=None, level_map=None, stream=None):
+    _check(lib().psa_attention_fwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(ws),
+                                   ws.numel(), _ptr(level_map), _ptr(O), _ptr(lse),
+                                   _stream(stream)), "psa_attention_fwd")
+
+
+def forward(p: Params, Q, K, V, O, ws, lse=None, level_map=None, stream=None):
+    _check(lib().psa_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                             _ptr(level_map), _ptr(ws), ws.numel(), _stream(stream)),
+           "psa_forward")
+
+
+def check_device(p: Params, ws: torch.Tensor, stream=None):
+    _check(lib().psa_check_device(ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
+           "psa_check_device")
+
+
+def map_shape(p: Params) -> Tuple[int, int, int, int]:
+    return (p.B, p.Hq, -(-p.N // p.q_blk), -(-p.N // p.kv_blk))
+
+
+def psa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_blk: int = 128,
+                kv_blk: int = 64, tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97),
+                causal: bool = False, forced_prefix_tokens: int = 0, scale: float = 0.0,
+                return_map: bool = False, workspace: Optional[torch.Tensor] = None):
+    """PSA forward on CUDA tensors q [B, Hq, N, d], k/v [B, Hkv, N, d]
+    (contiguous, bf16 or fp32).  Returns (O, lse) or (O, lse, level_map)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    p = make_params(B, Hq, Hkv, N, d, q_blk, kv_blk, tau, causal, forced_prefix_tokens, scale,
+                    q.dtype)
+    ws = workspace if workspace is not None else new_workspace(p, q.device)
+    O = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    lm = torch.empty(map_shape(p), dtype=torch.int8, device=q.device) if return_map else None
+    forward(p, q.contiguous(), k.contiguous(), v.contiguous(), O, ws, lse, lm)
+    return (O, lse, lm) if return_map else (O, lse)
+
+
+def workspace_layout(p: Params) -> dict:
+    """Byte offsets of the workspace regions (mirrors the library's layout),
+    for inspecting intermediate results."""
+    a256 = lambda x: (x + 255) & ~255
+    es = 2 if p.dtype == BF16 else 4
+    Nq, Nk = -(-p.N // p.q_blk), -(-p.N // p.kv_blk)
+    rows = [-(-p.N // (1 << l)) for l in range(4)]
+    off, L = 256, {"err": 0, "rows": rows, "Nq": Nq, "Nk": Nk, "kp": [0] * 4, "vp": [0] * 4}
+    for l in range(1, 4):
+        n = a256(p.B * p.Hkv * rows[l] * p.d * es)
+        L["kp"][l], off = off, off + n
+        L["vp"][l], off = off, off + n
+    L["k3f"], off = off, off + a256(p.B * p.Hkv * rows[3] * p.d * 4)
+    rq = p.B * p.Hq * Nq
+    L["qmean"], off = off, off + a256(rq * p.d * 4)
+    L["zlog"], off = off, off + a256(rq * Nk * 4)
+    L["map"], off = off, off + a256(rq * Nk)
+    L["counts"], off = off, off + a256(rq * 16)
+    L["list"], off = off, off + a256(rq * Nk * 4)
+    L["total"] = off
+    return L
+
+
+def workspace_view(ws: torch.Tensor, offset: int, shape, dtype: torch.dtype) -> torch.Tensor:
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    return ws[offset:offset + nbytes].view(dtype).view(*shape)

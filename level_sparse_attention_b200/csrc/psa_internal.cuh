@@ -1,0 +1,119 @@
+// Internal definitions shared by the PSA kernels and the C-ABI layer:
+// workspace layout, launch descriptions, small device helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/psa.h"
+
+namespace psa {
+
+constexpr int kLevels = 4;
+constexpr int kMaxNk = 8192;          // KV blocks per query block row (N <= 524288 at 64)
+constexpr int kErrTimeout = 1;        // bit in the device error word
+
+inline __host__ __device__ size_t cdiv(size_t a, size_t b) { return (a + b - 1) / b; }
+inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Byte offsets of everything kept in the caller's workspace.
+struct Layout {
+  size_t err;                 // int32 device error word (+ padding)
+  size_t kp[kLevels];         // pooled keys, level 1..3 (index 0 unused)
+  size_t vp[kLevels];         // pooled values, level 1..3
+  size_t k3f;                 // level-3 keys in fp32 [B, Hkv, ceil(N/8), d]
+  size_t qmean;               // query-block means fp32 [B, Hq, Nq, d]
+  size_t zlog;                // block logits fp32 [B, Hq, Nq, Nk]
+  size_t map;                 // internal level map int8 [B, Hq, Nq, Nk]
+  size_t counts;              // int4 per query block: entries at level 0..3
+  size_t list;                // int32 [B, Hq, Nq, Nk]: KV block indices, by level then index
+  size_t total;
+  size_t rows[kLevels];       // rows per head of each level
+  int Nq, Nk;
+};
+
+inline __host__ __device__ Layout make_layout(const psa_params_t& p) {
+  Layout L;
+  const size_t es = p.dtype == PSA_BF16 ? 2 : 4;
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.Nq = (int)cdiv(p.N, p.q_blk);
+  L.Nk = (int)cdiv(p.N, p.kv_blk);
+  for (int l = 0; l < kLevels; ++l) L.rows[l] = cdiv(p.N, (size_t)1 << l);
+  L.kp[0] = L.vp[0] = 0;
+  for (int l = 1; l < kLevels; ++l) {
+    const size_t bytes = align256((size_t)p.B * p.Hkv * L.rows[l] * p.d * es);
+    L.kp[l] = off; off += bytes;
+    L.vp[l] = off; off += bytes;
+  }
+  L.k3f = off; off += align256((size_t)p.B * p.Hkv * L.rows[3] * p.d * 4);
+  const size_t rowsq = (size_t)p.B * p.Hq * L.Nq;
+  L.qmean = off; off += align256(rowsq * p.d * 4);
+  L.zlog = off; off += align256(rowsq * L.Nk * 4);
+  L.map = off; off += align256(rowsq * L.Nk);
+  L.counts = off; off += align256(rowsq * 16);
+  L.list = off; off += align256(rowsq * L.Nk * 4);
+  L.total = off;
+  return L;
+}
+
+// Launch description passed by value to the mask-stage kernels.
+struct MaskArgs {
+  int B, Hq, Hkv, N, d, q_blk, kv_blk, Nq, Nk;
+  int causal, forced_prefix_tokens;
+  float scale;
+  float tau[kLevels];
+};
+
+inline MaskArgs make_mask_args(const psa_params_t& p, const Layout& L, float scale) {
+  MaskArgs a;
+  a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.N = p.N; a.d = p.d;
+  a.q_blk = p.q_blk; a.kv_blk = p.kv_blk; a.Nq = L.Nq; a.Nk = L.Nk;
+  a.causal = p.causal; a.forced_prefix_tokens = p.forced_prefix_tokens;
+  a.scale = scale;
+  for (int l = 0; l < kLevels; ++l) a.tau[l] = p.tau[l];
+  return a;
+}
+
+// ----------------------------------------------------------------- device
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+}  // namespace psa
+
+// Host-side launchers implemented in the kernel files.
+namespace psa {
+cudaError_t launch_pyramid(const psa_params_t& p, const Layout& L, const void* K, const void* V,
+                           char* ws, cudaStream_t st);
+cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, char* ws,
+                         cudaStream_t st);
+cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, char* ws,
+                         cudaStream_t st);
+cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, char* ws,
+                          int8_t* user_map, float* block_mass, cudaStream_t st);
+cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int8_t* map,
+                               char* ws, cudaStream_t st);
+cudaError_t launch_attention_simt(const psa_params_t& p, const Layout& L, float scale,
+                                  const void* Q, const void* K, const void* V, const char* ws,
+                                  void* O, float* lse, cudaStream_t st);
+bool attention_tc_supported(const psa_params_t& p);
+cudaError_t launch_attention_tc(const psa_params_t& p, const Layout& L, float scale,
+                                const void* Q, const void* K, const void* V, char* ws,
+                                void* O, float* lse, cudaStream_t st);
+}  // namespace psa

@@ -1,0 +1,83 @@
+"""The C ABI on the host: the library loads, exports every entry point that
+include/psa.h declares, and rejects bad arguments before launching anything.
+No GPU needed (no call here reaches a kernel launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import level_sparse_attention_b200 as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "psa.h")).read()
+    return sorted(set(re.findall(r"^\S.*?\b(psa_\w+)\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_entry_point():
+    L = P.lib()
+    names = header_functions()
+    assert set(names) == set(P.EXPORTED), names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_workspace_layout_matches_library():
+    for w in [(1, 12, 12, 32760, 128, 128, torch.bfloat16), (1, 2, 2, 1024, 64, 64, torch.float32),
+              (2, 28, 4, 16384, 128, 128, torch.bfloat16), (1, 3, 1, 77, 64, 128, torch.bfloat16)]:
+        B, Hq, Hkv, N, d, qb, dt = w
+        p = P.make_params(B, Hq, Hkv, N, d, q_blk=qb, dtype=dt)
+        assert P.workspace_layout(p)["total"] == P.workspace_size(p)
+
+
+@pytest.mark.parametrize("field,value", [
+    ("d", 96), ("d", 0), ("Hkv", 3), ("q_blk", 32), ("kv_blk", 128), ("N", 0), ("B", -1),
+    ("n_levels", 3), ("causal", 2), ("forced_prefix_tokens", -1), ("N", 64 * 8192 + 1)])
+def test_invalid_params_give_zero_workspace(field, value):
+    p = P.make_params(1, 10, 10, 4096, 128)
+    setattr(p, field, value)
+    assert P.workspace_size(p) == 0
+
+
+@pytest.mark.parametrize("tau", [(0.5, 0.4, 0.9, 0.95), (0.0, 0.5, 0.9, 0.95),
+                                 (0.5, 0.6, 0.9, 1.5), (float("nan"), 0.5, 0.9, 0.95)])
+def test_bad_thresholds_rejected(tau):
+    assert P.workspace_size(P.make_params(1, 2, 2, 1024, 64, tau=tau)) == 0
+
+
+def test_bad_pool_rejected():
+    p = P.make_params(1, 2, 2, 1024, 64)
+    p.pool[2] = 3
+    assert P.workspace_size(p) == 0
+
+
+def _call_forward(p, q, k, v, o, ws, nbytes):
+    return P.lib().psa_forward(ctypes.byref(p), q, k, v, o, None, None, ws, nbytes, None)
+
+
+def test_argument_errors_before_any_launch():
+    p = P.make_params(1, 2, 2, 1024, 64)
+    need = P.workspace_size(p)
+    A = ctypes.c_void_p(0x10000)            # aligned fake addresses: never dereferenced,
+    B = ctypes.c_void_p(0x20000)            # every call below fails validation first
+    mis = ctypes.c_void_p(0x10008)
+    assert _call_forward(p, None, A, A, A, B, need) == 1            # NULL Q
+    assert _call_forward(p, mis, A, A, A, B, need) == 3             # misaligned Q
+    assert _call_forward(p, A, A, A, A, B, need - 1) == 4           # workspace too small
+    assert _call_forward(p, A, A, A, A, ctypes.c_void_p(0x20010), need) == 3   # ws not 256-aligned
+    assert _call_forward(p, A, A, A, A, None, need) == 1
+    bad = P.make_params(1, 2, 2, 1024, 96)
+    assert _call_forward(bad, A, A, A, A, B, need) == 2             # d = 96 unsupported
+    assert P.lib().psa_build_pyramid(ctypes.byref(p), None, A, B, need, None) == 1
+    assert P.lib().psa_score_and_mask(ctypes.byref(p), A, B, need, None, mis, None) == 3
+    assert P.lib().psa_attention_fwd(ctypes.byref(p), A, A, A, B, need, None, A, mis, None) == 3
+
+
+def test_status_strings():
+    for s in range(7):
+        assert P.status_string(s)
+    assert "timeout" in P.status_string(6)

@@ -1,0 +1,88 @@
+"""Full-size workloads (the video-DiT and VLM shapes) through psa_forward, in
+the launch configuration the benchmark times.  The oracle checks sampled heads:
+the whole level map of each sampled head (with the near-threshold / near-tie
+exemptions) and the output rows of sampled query blocks, computed by the
+oracle on the map the GPU chose."""
+import numpy as np
+import pytest
+import torch
+
+import level_sparse_attention_b200 as P
+import oracle as O
+import workloads as W
+from tests import gpu_common as G
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+FULL = ["wan2.1_1.3b", "cogvideox_5b", "wan2.1_14b_720p", "qwen2.5_vl_7b"]
+
+
+def sample_heads(w):
+    hs = sorted({0, w.Hq // 2, w.Hq - 1})
+    return [(0, h) for h in hs]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    w = W.BY_NAME[name]
+    tau = W.thresholds(w)
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp, fused=True)
+    gm = run.level_map.cpu().numpy()
+    grp = w.Hq // w.Hkv
+    rng = np.random.default_rng(7)
+    total_thr = total_tie = 0
+    for b, h in sample_heads(w):
+        Q = inp.as_f64("q", b, h)
+        K, V = inp.as_f64("k", b, h // grp), inp.as_f64("v", b, h // grp)
+        pyr = O.build_pyramid(K, V)
+        s = 1.0 / np.sqrt(w.d)
+        z = O.block_logits(O.query_block_means(Q, w.q_blk), pyr, w.kv_blk, s)
+        mask = O.assign_levels(z, tau, w.N, w.q_blk, w.kv_blk, w.causal, w.forced_prefix_tokens)
+        unexplained, thr, tie = G.map_mismatch_report(gm[b, h], mask, tau)
+        assert unexplained == 0, (name, h, unexplained, thr, tie)
+        total_thr += thr
+        total_tie += tie
+        # output rows of a few query blocks (first, last, random), oracle on the GPU's map
+        blocks = sorted({0, w.Nq - 1, int(rng.integers(0, w.Nq))})
+        sub = np.full_like(gm[b, h], -1)
+        sub[blocks] = gm[b, h][blocks]
+        ref_O, ref_lse = O.pyramid_attention(Q, pyr, sub, w.q_blk, w.kv_blk, s, w.causal)
+        rows = np.concatenate([np.arange(a * w.q_blk, min((a + 1) * w.q_blk, w.N)) for a in blocks])
+        gO = G.to_f64(run.O[b, h])
+        G.compare_out(gO, ref_O, w.dtype, rows=rows)
+        G.compare_lse(run.lse[b, h].cpu().numpy().astype(np.float64)[rows], ref_lse[rows], w.dtype)
+    # every head: a row keeps at least its top block; rows never keep blocks after a causal row
+    assert np.all((gm >= 0).sum(-1) >= 1)
+    if w.causal:
+        for a in range(w.Nq):
+            last = min((a + 1) * w.q_blk, w.N) - 1
+            assert np.all(gm[:, :, a, last // w.kv_blk + 1:] == -1)
+    print(f"{name}: near-threshold {total_thr}, near-tie {total_tie} exempt mismatches")
+
+
+def test_max_size_single_head():
+    """Largest supported sequence (8192 KV blocks of 64: N = 524288), one head,
+    d = 64: the 8192-entry sort and the long work lists."""
+    base = W.BY_NAME["cogvideox_5b"]
+    w = W.with_overrides(base, Hq=1, Hkv=1, n_text=0, grid=(8, 256, 256), coarse=(2, 64, 64),
+                         forced_prefix_tokens=0, seed=31, target="fixed")
+    assert w.N == 524288 and w.Nk == 8192
+    tau = (0.02, 0.03, 0.04, 0.05)
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp, tau=tau, fused=True)
+    gm = run.level_map.cpu().numpy()[0, 0]
+    Q, K, V = inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0), inp.as_f64("v", 0, 0)
+    pyr = O.build_pyramid(K, V)
+    s = 1.0 / np.sqrt(w.d)
+    qb = O.query_block_means(Q, w.q_blk)
+    blocks = [0, 1777, w.Nq - 1]
+    z = O.block_logits(qb[blocks], pyr, w.kv_blk, s)
+    mask = O.assign_levels(z, tau, w.N, w.q_blk, w.kv_blk)
+    unexplained, _, _ = G.map_mismatch_report(gm[blocks], mask, tau)
+    assert unexplained == 0
+    sub = np.full_like(gm, -1)
+    sub[blocks] = gm[blocks]
+    ref_O, _ = O.pyramid_attention(Q, pyr, sub, w.q_blk, w.kv_blk, s)
+    rows = np.concatenate([np.arange(a * w.q_blk, min((a + 1) * w.q_blk, w.N)) for a in blocks])
+    G.compare_out(G.to_f64(run.O[0, 0]), ref_O, w.dtype, rows=rows)

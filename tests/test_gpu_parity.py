@@ -1,0 +1,170 @@
+"""GPU parity of every stage of the PSA forward pass against the CPU oracle,
+through the C ABI, at sizes the oracle finishes in seconds (several tiles and
+ragged tails in every case)."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import level_sparse_attention_b200 as P
+import oracle as O
+import workloads as W
+from tests import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+BASE = W.BY_NAME
+CASES = {
+    # the tiny fp32 workload as specified (64-row query blocks, CUDA-core path)
+    "tiny_f32": BASE["tiny_f32"],
+    # tensor-core path, d = 128, ragged N = 1000 (last query block 104 rows, last KV block 40)
+    "bf16_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, grid=(1, 20, 50),
+                                  coarse=(1, 5, 13), seed=11, target="fixed"),
+    # tensor-core path, d = 64, text prefix forced to level 0, N = 226 + 760
+    "bf16_d64_text": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, grid=(1, 20, 38),
+                                      coarse=(1, 5, 10), seed=12, target="fixed"),
+    # grouped queries (2 per KV head), causal, N = 1000
+    "bf16_gqa_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=4, Hkv=2, grid=(1, 25, 40),
+                                        coarse=(1, 7, 10), seed=13, target="fixed"),
+    # CUDA-core path for bf16 with 64-row query blocks, causal
+    "bf16_q64_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 20, 33),
+                                        coarse=(1, 5, 9), seed=14, q_blk=64, target="fixed"),
+    # CUDA-core path, fp32, d = 128, 128-row query blocks
+    "f32_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, dtype="f32",
+                                 grid=(1, 18, 40), coarse=(1, 5, 10), seed=15, target="fixed"),
+}
+
+_cache = {}
+
+
+def setup(name):
+    if name not in _cache:
+        w = CASES[name]
+        inp = W.make_inputs(w)
+        heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+        ref = G.oracle_heads(w, inp, heads)
+        run = G.run_stages(w, inp)
+        _cache[name] = (w, inp, ref, run)
+    return _cache[name]
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_pyramid_levels(name):
+    w, inp, _, run = setup(name)
+    L = P.workspace_layout(run.p)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    for hk in range(w.Hkv):
+        pyr = O.build_pyramid(inp.as_f64("k", 0, hk), inp.as_f64("v", 0, hk))
+        for l in range(1, 4):
+            shape = (w.B, w.Hkv, L["rows"][l], w.d)
+            for key, ref in (("kp", pyr.keys[l]), ("vp", pyr.values[l])):
+                got = G.to_f64(run.view(key, shape, tdt, l)[0, hk])
+                tol = (2.0 ** -8 if w.dtype == "bf16" else 1e-6) * np.abs(ref) + 1e-6
+                assert np.all(np.abs(got - ref) <= tol), (key, l, np.abs(got - ref).max())
+        k3 = G.to_f64(run.view("k3f", (w.B, w.Hkv, L["rows"][3], w.d), torch.float32)[0, hk])
+        assert np.abs(k3 - pyr.keys[3]).max() <= 1e-5
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_block_logits(name):
+    w, inp, ref, run = setup(name)
+    L = P.workspace_layout(run.p)
+    z = G.to_f64(run.view("zlog", (w.B, w.Hq, L["Nq"], L["Nk"]), torch.float32))
+    for (b, h), r in ref.items():
+        vis = np.array([[O.visible(a, j, w.N, w.q_blk, w.kv_blk, w.causal) for j in range(L["Nk"])]
+                        for a in range(L["Nq"])])
+        err = np.abs(z[b, h] - r.z)[vis]
+        assert err.max() <= 1e-4, err.max()
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_level_map(name):
+    w, inp, ref, run = setup(name)
+    gm = run.level_map.cpu().numpy()
+    tau = W.thresholds(w)
+    for (b, h), r in ref.items():
+        unexplained, thr, tie = G.map_mismatch_report(gm[b, h], r.mask, tau)
+        assert unexplained == 0, (b, h, unexplained, thr, tie)
+        mass = G.to_f64(run.mass[b, h])
+        assert np.abs(mass - r.mask.mass).max() <= 1e-5
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_work_list_matches_map(name):
+    w, inp, ref, run = setup(name)
+    L = P.workspace_layout(run.p)
+    Nq, Nk = L["Nq"], L["Nk"]
+    gm = run.level_map.cpu().numpy()
+    counts = run.view("counts", (w.B, w.Hq, Nq, 4), torch.int32).cpu().numpy()
+    lst = run.view("list", (w.B, w.Hq, Nq, Nk), torch.int32).cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.Hq):
+            for a in range(Nq):
+                want = [j for l in range(4) for j in range(Nk) if gm[b, h, a, j] == l]
+                n = [int((gm[b, h, a] == l).sum()) for l in range(4)]
+                assert counts[b, h, a].tolist() == n
+                assert lst[b, h, a, :len(want)].tolist() == want
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_attention_on_oracle_map(name):
+    """Attention alone: the kernel is fed the oracle's own map."""
+    w, inp, ref, _ = setup(name)
+    omap = np.zeros((w.B, w.Hq) + ref[(0, 0)].mask.level_map.shape, dtype=np.int8)
+    for (b, h), r in ref.items():
+        omap[b, h] = r.mask.level_map
+    run = G.run_stages(w, inp, external_map=omap)
+    gO, glse = G.to_f64(run.O), run.lse.cpu().numpy().astype(np.float64)
+    for (b, h), r in ref.items():
+        G.compare_out(gO[b, h], r.O, w.dtype)
+        G.compare_lse(glse[b, h], r.lse, w.dtype)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("kind", ["random", "all_level3", "all_level0", "pruned_rows", "binary"])
+def test_attention_on_external_maps(name, kind):
+    w, inp, _, _ = setup(name)
+    Nq, Nk = w.Nq, w.Nk
+    rng = np.random.default_rng(zlib.crc32(f"{name}/{kind}".encode()))
+    m = np.empty((w.B, w.Hq, Nq, Nk), dtype=np.int8)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            if kind == "random":
+                m[b, h] = G.rand_map(rng, Nq, Nk)
+            elif kind == "all_level3":
+                m[b, h] = 3
+            elif kind == "all_level0":
+                m[b, h] = 0
+            elif kind == "pruned_rows":
+                m[b, h] = G.rand_map(rng, Nq, Nk, 0, 4)
+                m[b, h, ::2] = -1
+            else:
+                m[b, h] = np.where(rng.random((Nq, Nk)) < 0.4, 0, -1)
+    run = G.run_stages(w, inp, external_map=m)
+    ref = G.oracle_heads(w, inp, [(0, h) for h in range(w.Hq)], level_map=m)
+    gO, glse = G.to_f64(run.O), run.lse.cpu().numpy().astype(np.float64)
+    for (b, h), r in ref.items():
+        G.compare_out(gO[b, h], r.O, w.dtype)
+        G.compare_lse(glse[b, h], r.lse, w.dtype)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fused_forward(name):
+    """psa_forward end to end; its attention is checked against the oracle's
+    attention on the map the GPU chose (map parity is checked above)."""
+    w, inp, ref, _ = setup(name)
+    run = G.run_stages(w, inp, fused=True)
+    gm = run.level_map.cpu().numpy()
+    tau = W.thresholds(w)
+    for (b, h), r in ref.items():
+        assert G.map_mismatch_report(gm[b, h], r.mask, tau)[0] == 0
+    ref_g = G.oracle_heads(w, inp, list(ref), level_map=gm)
+    gO = G.to_f64(run.O)
+    for (b, h), r in ref_g.items():
+        G.compare_out(gO[b, h], r.O, w.dtype)
+
+
+def test_no_device_timeouts_recorded():
+    w, inp, _, run = setup("bf16_d128")
+    P.check_device(run.p, run.ws)
