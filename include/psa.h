@@ -132,6 +132,31 @@ psa_status_t psa_forward(const psa_params_t* params, const void* Q, const void* 
                          void* O, float* lse, int8_t* level_map, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Allocation-free forward pass.  The paper has no counterpart: this entry
+ * point exists for callers that may not allocate device memory while they
+ * run, such as a host framework that plans all memory ahead and hands a plugin
+ * only its inputs and outputs, or a latency-sensitive loop that cannot afford
+ * the device-wide synchronisation of cudaMalloc/cudaFree.  It does exactly
+ * what psa_forward does, with the same arguments minus the workspace: the
+ * scratch comes from a 32 MiB device array inside the library, held on every
+ * GPU that loads the library until the process exits.
+ *  - Returns PSA_ERR_WORKSPACE_TOO_SMALL, launching nothing, when
+ *    psa_workspace_size(params) exceeds 32 MiB; invalid parameters give the
+ *    same status as psa_forward.
+ *  - Allocates nothing (no cudaMalloc/cudaFree); it clears the array's error
+ *    word with cudaMemsetAsync on `stream`, then enqueues psa_forward's kernels.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call uses the same array, which keeps the previous call's contents:
+ *    calls that overlap on the GPU (other streams, unordered host threads)
+ *    race and give wrong results.  Serialise them.
+ *  - A device timeout is recorded in the array's error word, which the next
+ *    call clears; psa_check_device cannot read it. */
+psa_status_t psa_forward_noalloc(const psa_params_t* params, const void* Q, const void* K,
+                                 const void* V, void* O, float* lse, int8_t* level_map,
+                                 void* stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
  * check, PSA_ERR_CUDA if the stream reported an error, else PSA_OK. */

@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "psa_attention_fwd": (ctypes.c_int, [P, vp, vp, vp, vp, sz, vp, vp, vp, vp]),
             "psa_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "psa_check_device": (ctypes.c_int, [P, vp, sz, vp]),
+            "psa_forward_noalloc": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp]),
             "psa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sigs.items():
@@ -68,7 +69,8 @@ def lib() -> ctypes.CDLL:
 
 
 EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
-            "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string")
+            "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string",
+            "psa_forward_noalloc")
 
 
 def status_string(status: int) -> str:
@@ -141,6 +143,14 @@ def forward(p: Params, Q, K, V, O, ws, lse=None, level_map=None, stream=None):
     _check(lib().psa_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
                              _ptr(level_map), _ptr(ws), ws.numel(), _stream(stream)),
            "psa_forward")
+
+
+def forward_noalloc(p: Params, Q, K, V, O, lse=None, level_map=None, stream=None):
+    """psa_forward without a workspace: the library's own 32 MiB device array
+    serves as scratch (no allocation; calls must not overlap on the GPU)."""
+    _check(lib().psa_forward_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                     _ptr(lse), _ptr(level_map), _stream(stream)),
+           "psa_forward_noalloc")
 
 
 def check_device(p: Params, ws: torch.Tensor, stream=None):

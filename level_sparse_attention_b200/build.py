@@ -9,7 +9,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["pyramid.cu", "mask.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu"]
+SOURCES = ["pyramid.cu", "mask.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu",
+           "psa_noalloc.cu"]
 LIB = os.path.join(HERE, "libpsa.so")
 
 
