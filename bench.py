@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-heads", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling aid: run only this many query heads (KV heads scaled to match)")
     return ap.parse_args()
 
 
@@ -160,6 +162,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = W.BY_NAME[args.workload]
     tau = W.thresholds(w)
+    if args.heads:
+        grp = w.Hq // w.Hkv
+        w = W.with_overrides(w, Hq=args.heads, Hkv=max(1, args.heads // grp))
     p = P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk, tau, w.causal,
                       w.forced_prefix_tokens, 0.0,
                       torch.bfloat16 if w.dtype == "bf16" else torch.float32)

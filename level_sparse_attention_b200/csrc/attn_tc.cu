@@ -45,15 +45,17 @@ constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
 template <int D>
 struct Cfg {
   static constexpr int HALVES = D / 64;
-  static constexpr int STAGES = D == 128 ? 2 : 4;
-  static constexpr int HALF = kBN * 128;            // bytes of one 64-column half tile
+  static constexpr int KSTAGES = D == 128 ? 3 : 6;   // K ring (freed when QK^T completes)
+  static constexpr int VSTAGES = D == 128 ? 2 : 4;   // V ring (freed when PV completes)
+  static constexpr int MSTAGES = 4;                  // per-tile bias / position tables
+  static constexpr int HALF = kBN * 128;             // bytes of one 64-column half tile
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int KV_BYTES = kBN * D * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_META = OFF_V + STAGES * KV_BYTES;    // per stage: bias[128], kpos[128]
-  static constexpr int OFF_BAR = OFF_META + STAGES * 1024;
+  static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
+  static constexpr int OFF_META = OFF_V + VSTAGES * KV_BYTES;   // per table: bias[128], kpos[128]
+  static constexpr int OFF_BAR = OFF_META + MSTAGES * 1024;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;             // + slack for 1024 alignment
 };
 
@@ -66,7 +68,7 @@ struct __align__(64) TcParams {
   __nv_bfloat16* O;
   float* lse;
   int* err;
-  int Hq, Hkv, N, Nq, Nk, causal;
+  int Hq, Hkv, N, Nq, Nk, causal, n_rows;
   float scale_log2;
 };
 
@@ -128,6 +130,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -235,7 +243,31 @@ __device__ __forceinline__ RowWork row_work(int4 c) {
   return w;
 }
 
-// ------------------------------------------------------------------ kernel
+// The entries of tile t, one per lane: lane i takes entry e0 + i.  Entries
+// never cross a tile edge, so the lanes inside the tile form a prefix.
+struct TileEntry {
+  bool in_tile;
+  int j, l, R, r0;          // KV block, level, sub-block rows, first row in the tile
+};
+
+__device__ __forceinline__ TileEntry tile_entry(const RowWork& w, const int* lrow, int e0, int t,
+                                                int lane) {
+  TileEntry te;
+  const int e = e0 + lane;
+  int l = 0;
+  while (l < kLevels - 1 && e >= w.first[l + 1]) ++l;
+  te.l = l;
+  te.R = 64 >> l;
+  const int off = w.base[l] + (e - w.first[l]) * te.R;
+  te.in_tile = e < w.first[kLevels] && off < (t + 1) * kBN;
+  te.r0 = off - t * kBN;
+  te.j = te.in_tile ? __ldg(lrow + e) : 0;
+  return te;
+}
+
+// Items (query blocks) of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+// Consecutive CTAs take consecutive query blocks of the same head, so the
+// head's K/V and pyramid stay in L2 while its query blocks are processed.
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -245,30 +277,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  // barrier slots
-  const int B_QFULL = 0, B_KFULL = 1, B_VFULL = 1 + C::STAGES, B_EMPTY = 1 + 2 * C::STAGES;
-  const int B_SFULL = 1 + 3 * C::STAGES, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
-  const int B_FINAL = B_ODONE + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_FINAL + 1);
+  constexpr int KS = C::KSTAGES, VS = C::VSTAGES, MS = C::MSTAGES;
+  constexpr int B_QFULL = 0, B_QEMPTY = 1;
+  constexpr int B_KFULL = 2, B_KEMPTY = B_KFULL + KS;
+  constexpr int B_VFULL = B_KEMPTY + KS, B_VEMPTY = B_VFULL + VS;
+  constexpr int B_MFULL = B_VEMPTY + VS, B_MEMPTY = B_MFULL + MS;
+  constexpr int B_SFULL = B_MEMPTY + MS, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
+  constexpr int B_FINAL = B_ODONE + 2, NBARS = B_FINAL + 1;
+  static_assert(NBARS * 8 + 16 <= 512, "barrier area");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row_id = blockIdx.x;                 // (b*Hq + hq) * Nq + qa
-  const int qa = row_id % p.Nq;
-  const int bhq = row_id / p.Nq;
-  const int b = bhq / p.Hq, hq = bhq % p.Hq;
-  const int bhk = b * p.Hkv + hq / (p.Hq / p.Hkv);
-  const RowWork w = row_work(p.counts[row_id]);
-  const int T = w.tiles;
+  const int n_items = p.n_rows;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_EMPTY + s), 1);
-    }
+    mbar_init(bar(B_QEMPTY), 1);
+    for (int s = 0; s < KS; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
+    for (int s = 0; s < VS; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
+    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 1); mbar_init(bar(B_MEMPTY + s), 4); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
       mbar_init(bar(B_PFULL + i), 128);
@@ -278,11 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // Zero the K/V stages once: rows of a partial last tile are never loaded, and
+  // Zero the K/V rings once: rows of a partial last tile are never loaded, and
   // their (masked, P = 0) products must not meet NaN bit patterns.
   {
     uint4* kv = reinterpret_cast<uint4*>(smem + C::OFF_K);
-    const int n16 = (2 * C::STAGES * C::KV_BYTES) / 16;
+    const int n16 = (C::OFF_META - C::OFF_K) / 16;
     for (int i = threadIdx.x; i < n16; i += kThreads) kv[i] = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -301,109 +330,142 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (T > 0) {
+    int gk = 0, gv = 0, iq = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+      const RowWork w = row_work(p.counts[item]);
+      const int T = w.tiles;
+      if (T == 0) continue;
+      const int qa = item % p.Nq, bhq = item / p.Nq;
+      const int bhk = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / (p.Hq / p.Hkv);
+      const int* lrow = p.list + (long long)item * p.Nk;
+      if (iq > 0 && !warp_wait(bar(B_QEMPTY), (iq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
       if (lane == 0) {
         mbar_expect_tx(bar(B_QFULL), C::Q_BYTES);
         for (int h = 0; h < C::HALVES; ++h)
           tma_load_3d(sbase + C::OFF_Q + h * (kBM * 128), &p.tq, bar(B_QFULL), h * 64,
                       qa * kBM, bhq);
       }
-      const int* lrow = p.list + (long long)row_id * p.Nk;
-      int e_next = 0;
-      for (int t = 0; t < T; ++t) {
-        const int s = t % C::STAGES;
-        if (t >= C::STAGES &&
-            !warp_wait(bar(B_EMPTY + s), ((t / C::STAGES) + 1) & 1, abort_flag, p.err))
-          break;
-        float* mbias = reinterpret_cast<float*>(smem + C::OFF_META + s * 1024);
-        int* mpos = reinterpret_cast<int*>(mbias + kBN);
-        const int e = e_next + lane;
-        int l = 0;
-        while (l < kLevels - 1 && e >= w.first[l + 1]) ++l;
-        const int R = 64 >> l;
-        const int off = w.base[l] + (e - w.first[l]) * R;
-        const bool in_tile = e < w.first[kLevels] && off < (t + 1) * kBN;
-        int j = 0, r0 = 0;
-        if (in_tile) {
-          j = lrow[e];
-          r0 = off - t * kBN;
-          const long long g0 = (long long)j * R;      // first level-l row of block j
-          for (int rr = 0; rr < R; ++rr) {
-            const long long g = g0 + rr;
-            const long long tok = g << l;
-            const int cg = (int)min((long long)(1 << l), (long long)p.N - tok);
-            mbias[r0 + rr] = cg > 0 ? log2f((float)cg) : -INFINITY;
-            mpos[r0 + rr] = (p.causal && l == 0) ? (int)tok : INT_MIN;
-          }
-        }
-        const unsigned ballot = __ballot_sync(0xffffffffu, in_tile);
-        const int n_in = __popc(ballot);
-        if (t == T - 1) {      // keys after the last entry: no key
-          for (int c = w.base[kLevels] - t * kBN + lane; c < kBN; c += 32) {
-            if (c >= 0) {
-              mbias[c] = -INFINITY;
-              mpos[c] = INT_MIN;
-            }
-          }
-        }
-        int bytes = in_tile ? R * D * 2 : 0;
+      ++iq;
+      int ek = 0, ev = 0;
+      for (int t = 0; t <= T; ++t) {
+        if (t < T) {
+          // K of tile t, and its per-key bias / position table
+          const int s = gk % KS, ms = gk % MS;
+          if (gk >= KS && !warp_wait(bar(B_KEMPTY + s), ((gk / KS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (gk >= MS && !warp_wait(bar(B_MEMPTY + ms), ((gk / MS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          const TileEntry te = tile_entry(w, lrow, ek, t, lane);
+          const unsigned ballot = __ballot_sync(0xffffffffu, te.in_tile);
+          const int n_in = __popc(ballot);
+          int bytes = te.in_tile ? te.R * D * 2 : 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-        __threadfence_block();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_expect_tx(bar(B_KFULL + s), bytes);
-          mbar_expect_tx(bar(B_VFULL + s), bytes);
+          for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+          // table: lane covers columns 4*lane .. 4*lane+3 (inside one 8-column chunk)
+          const int col = 4 * lane;
+          int owner = 0;
+          for (int i = 1; i < n_in; ++i)
+            if (__shfl_sync(0xffffffffu, te.r0, i) <= col) owner = i;
+          const int oj = __shfl_sync(0xffffffffu, te.j, owner);
+          const int ol = __shfl_sync(0xffffffffu, te.l, owner);
+          const int oR = __shfl_sync(0xffffffffu, te.R, owner);
+          const int or0 = __shfl_sync(0xffffffffu, te.r0, owner);
+          const bool live = n_in > 0 && col < or0 + oR;   // false past the last entry
+          float bias[4];
+          int kpos[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const long long g = (long long)oj * oR + (col + c - or0);
+            const long long tok = g << ol;
+            const int cnt = (int)min((long long)(1 << ol), (long long)p.N - tok);
+            bias[c] = !live || cnt <= 0 ? -INFINITY : (cnt == (1 << ol) ? (float)ol : log2f((float)cnt));
+            kpos[c] = (live && p.causal && ol == 0) ? (int)tok : INT_MIN;
+          }
+          float* mb = reinterpret_cast<float*>(smem + C::OFF_META + ms * 1024);
+          reinterpret_cast<float4*>(mb)[lane] = make_float4(bias[0], bias[1], bias[2], bias[3]);
+          reinterpret_cast<int4*>(mb + kBN)[lane] = make_int4(kpos[0], kpos[1], kpos[2], kpos[3]);
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar(B_MFULL + ms));
+            mbar_expect_tx(bar(B_KFULL + s), bytes);
+          }
+          __syncwarp();
+          if (te.in_tile) {
+            const uint32_t kdst = sbase + C::OFF_K + s * C::KV_BYTES + te.r0 * 128;
+            for (int h = 0; h < C::HALVES; ++h)
+              tma_load_3d(kdst + h * C::HALF, &p.tk[te.l], bar(B_KFULL + s), h * 64, te.j * te.R, bhk);
+          }
+          ek += n_in;
+          ++gk;
         }
-        __syncwarp();
-        if (in_tile) {
-          const uint32_t kdst = sbase + C::OFF_K + s * C::KV_BYTES + r0 * 128;
-          const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + r0 * 128;
-          for (int h = 0; h < C::HALVES; ++h)
-            tma_load_3d(kdst + h * C::HALF, &p.tk[l], bar(B_KFULL + s), h * 64, j * R, bhk);
-          for (int h = 0; h < C::HALVES; ++h)
-            tma_load_3d(vdst + h * C::HALF, &p.tv[l], bar(B_VFULL + s), h * 64, j * R, bhk);
+        if (t >= 1) {
+          // V of tile t - 1
+          const int s = gv % VS;
+          if (gv >= VS && !warp_wait(bar(B_VEMPTY + s), ((gv / VS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          const TileEntry te = tile_entry(w, lrow, ev, t - 1, lane);
+          const int n_in = __popc(__ballot_sync(0xffffffffu, te.in_tile));
+          int bytes = te.in_tile ? te.R * D * 2 : 0;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+          if (lane == 0) mbar_expect_tx(bar(B_VFULL + s), bytes);
+          __syncwarp();
+          if (te.in_tile) {
+            const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + te.r0 * 128;
+            for (int h = 0; h < C::HALVES; ++h)
+              tma_load_3d(vdst + h * C::HALF, &p.tv[te.l], bar(B_VFULL + s), h * 64, te.j * te.R, bhk);
+          }
+          ev += n_in;
+          ++gv;
         }
-        e_next += n_in;
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
-    if (lane == 0 && T > 0) {
+    if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_bf16(kBM, kBN, false);
       constexpr uint32_t ID_PV = idesc_bf16(kBM, D, true);
-      bool ok = wait_bar(bar(B_QFULL), 0, abort_flag, p.err);
-      auto issue_pv = [&](int u) -> bool {
-        const int s = u % C::STAGES, bb = u & 1;
+      bool ok = true;
+      auto issue_pv = [&](int u, bool first) -> bool {
+        const int s = u % VS, bb = u & 1;
         if (!wait_bar(bar(B_PFULL + bb), (u >> 1) & 1, abort_flag, p.err)) return false;
-        if (!wait_bar(bar(B_VFULL + s), (u / C::STAGES) & 1, abort_flag, p.err)) return false;
+        if (!wait_bar(bar(B_VFULL + s), (u / VS) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
         const uint32_t vb = sbase + C::OFF_V + s * C::KV_BYTES;
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k)
           mma_ts(T_O, T_P + bb * 64 + k * 8, sdesc(vb + k * 2048, C::HALF, 1024), ID_PV,
-                 (u > 0 || k > 0) ? 1u : 0u);
+                 (first && k == 0) ? 0u : 1u);
         mma_commit(bar(B_ODONE + bb));
-        mma_commit(bar(B_EMPTY + s));
+        mma_commit(bar(B_VEMPTY + s));
         return true;
       };
-      for (int t = 0; ok && t < T; ++t) {
-        const int s = t % C::STAGES, bb = t & 1;
-        if (!wait_bar(bar(B_KFULL + s), (t / C::STAGES) & 1, abort_flag, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sbase + C::OFF_K + s * C::KV_BYTES;
-        const uint32_t qb = sbase + C::OFF_Q;
+      int g = 0, iq = 0;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const int T = row_work(p.counts[item]).tiles;
+        if (T == 0) continue;
+        if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
+        ++iq;
+        for (int t = 0; t < T; ++t) {
+          const int gk = g + t, s = gk % KS, bb = gk & 1;
+          if (!wait_bar(bar(B_KFULL + s), (gk / KS) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = sbase + C::OFF_K + s * C::KV_BYTES;
+          const uint32_t qb = sbase + C::OFF_Q;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t koff = (k >> 2) * C::HALF + (k & 3) * 32;
-          const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
-          mma_ss(T_S + bb * 128, sdesc(qb + qoff, 16, 1024), sdesc(kb + koff, 16, 1024), ID_QK,
-                 k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t koff = (k >> 2) * C::HALF + (k & 3) * 32;
+            const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
+            mma_ss(T_S + bb * 128, sdesc(qb + qoff, 16, 1024), sdesc(kb + koff, 16, 1024), ID_QK,
+                   k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(B_SFULL + bb));
+          mma_commit(bar(B_KEMPTY + s));
+          if (t == T - 1) mma_commit(bar(B_QEMPTY));
+          if (t >= 1 && !issue_pv(gk - 1, t == 1)) { ok = false; break; }
         }
-        mma_commit(bar(B_SFULL + bb));
-        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+        if (!ok || !issue_pv(g + T - 1, T == 1)) { ok = false; break; }
+        g += T;
       }
-      if (ok) issue_pv(T - 1);
       // drain: every MMA issued so far completes before TMEM is released
       mma_commit(bar(B_FINAL));
       const uint64_t t0 = global_ns();
@@ -414,109 +476,130 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // --------------------------------------------------------------- softmax
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int qpos = qa * kBM + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float m = -INFINITY, lsum = 0.f;
+    int g = 0;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int s = t % C::STAGES, bb = t & 1;
-      if (!warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, abort_flag, p.err) ||
-          !warp_wait(bar(B_KFULL + s), (t / C::STAGES) & 1, abort_flag, p.err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float* mbias = reinterpret_cast<const float*>(smem + C::OFF_META + s * 1024);
-      const int* mpos = reinterpret_cast<const int*>(mbias + kBN);
-      float x[kBN];
-#pragma unroll
-      for (int c0 = 0; c0 < kBN; c0 += 32)
-        tmem_ld32(T_S + bb * 128 + lane_off + c0, reinterpret_cast<uint32_t*>(x + c0));
-      tmem_ld_wait();
-      reg_fence<kBN>(reinterpret_cast<uint32_t*>(x));
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        float v = fmaf(x[c], p.scale_log2, mbias[c]);
-        if (p.causal && qpos < mpos[c]) v = -INFINITY;
-        x[c] = v;
-        mt = fmaxf(mt, v);
-      }
-      const float m_new = fmaxf(m, mt);
-      const bool need = m_new > m + kRescaleLog2;     // false while both are -inf
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_use = need ? m_new : m;
-        const float factor = need ? exp2f(m - m_use) : 1.f;   // 0 when m = -inf
-        if (t > 0) {
-          if (!warp_wait(bar(B_ODONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(T_O + lane_off + c0, o);
-            tmem_ld_wait();
-            reg_fence<32>(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-            tmem_st32(T_O + lane_off + c0, o);
-          }
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const int T = row_work(p.counts[item]).tiles;
+      const int qa = item % p.Nq, bhq = item / p.Nq;
+      const int qpos = qa * kBM + r;
+      float m = -INFINITY, lsum = 0.f;
+      for (int t = 0; ok && t < T; ++t) {
+        const int gt = g + t, bb = gt & 1, ms = gt % MS;
+        if (!warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) ||
+            !warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
         }
-        lsum *= factor;
-        m = m_use;
-      }
-      const float m_base = m == -INFINITY ? 0.f : m;
-      uint32_t pk[kBN / 2];
+        tc_fence_after();
+        const float* mbias = reinterpret_cast<const float*>(smem + C::OFF_META + ms * 1024);
+        const int* mpos = reinterpret_cast<const int*>(mbias + kBN);
+        float x[kBN];
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = exp2f(x[c] - m_base);
-        const float p1 = exp2f(x[c + 1] - m_base);
-        lsum += p0 + p1;
-        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-        pk[c / 2] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      tmem_st32(T_P + bb * 64 + lane_off, pk);
-      tmem_st32(T_P + bb * 64 + lane_off + 32, pk + 32);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + bb));
-    }
-    // epilogue
-    const bool row_ok = qpos < p.N;
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D;
-    const bool have_o = __all_sync(0xffffffffu, ok) && T > 0 &&
-                        warp_wait(bar(B_ODONE + ((T - 1) & 1)), ((T - 1) >> 1) & 1, abort_flag,
-                                  p.err);
-    if (have_o) tc_fence_after();
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(T_O + lane_off + c0, o);
+        for (int c0 = 0; c0 < kBN; c0 += 32)
+          tmem_ld32(T_S + bb * 128 + lane_off + c0, reinterpret_cast<uint32_t*>(x + c0));
         tmem_ld_wait();
-        reg_fence<32>(o);
-      } else {
+        reg_fence<kBN>(reinterpret_cast<uint32_t*>(x));
+        float mt = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      if (row_ok) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
-                                                   __uint_as_float(o[2 * i + 1]) * inv);
-          pk[i] = *reinterpret_cast<uint32_t*>(&h);
+        for (int c = 0; c < kBN; c += 4) {
+          const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
+          x[c] = fmaf(x[c], p.scale_log2, b4.x);
+          x[c + 1] = fmaf(x[c + 1], p.scale_log2, b4.y);
+          x[c + 2] = fmaf(x[c + 2], p.scale_log2, b4.z);
+          x[c + 3] = fmaf(x[c + 3], p.scale_log2, b4.w);
+          if (p.causal) {
+            const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
+            if (qpos < k4.x) x[c] = -INFINITY;
+            if (qpos < k4.y) x[c + 1] = -INFINITY;
+            if (qpos < k4.z) x[c + 2] = -INFINITY;
+            if (qpos < k4.w) x[c + 3] = -INFINITY;
+          }
+          mt = fmaxf(mt, fmaxf(fmaxf(x[c], x[c + 1]), fmaxf(x[c + 2], x[c + 3])));
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
+        const float m_new = fmaxf(m, mt);
+        const bool need = m_new > m + kRescaleLog2;     // false while both are -inf
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_use = need ? m_new : m;
+          const float factor = need ? ex2(m - m_use) : 1.f;   // 0 when m = -inf
+          if (t > 0) {
+            if (!warp_wait(bar(B_ODONE + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(T_O + lane_off + c0, o);
+              tmem_ld_wait();
+              reg_fence<32>(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+              tmem_st32(T_O + lane_off + c0, o);
+            }
+          }
+          lsum *= factor;
+          m = m_use;
+        }
+        const float m_base = m == -INFINITY ? 0.f : m;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2(x[h * 64 + c] - m_base);
+            const float p1 = ex2(x[h * 64 + c + 1] - m_base);
+            lsum += p0 + p1;
+            __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+            pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
+          }
+          tmem_st32(T_P + bb * 64 + lane_off + h * 32, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + bb));
       }
+      // epilogue of this query block
+      const bool row_ok = qpos < p.N;
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D;
+      const bool have_o = __all_sync(0xffffffffu, ok) && T > 0 &&
+                          warp_wait(bar(B_ODONE + ((g + T - 1) & 1)), ((g + T - 1) >> 1) & 1,
+                                    abort_flag, p.err);
+      if (have_o) tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(T_O + lane_off + c0, o);
+          tmem_ld_wait();
+          reg_fence<32>(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
+                                                      __uint_as_float(o[2 * i + 1]) * inv);
+            pk[i] = *reinterpret_cast<uint32_t*>(&hh);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (row_ok && p.lse)
+        p.lse[(long long)bhq * p.N + qpos] = lsum > 0.f ? (m + log2f(lsum)) * kLn2 : -INFINITY;
+      g += T;
+      if (!ok) break;
     }
-    if (row_ok && p.lse)
-      p.lse[(long long)bhq * p.N + qpos] = lsum > 0.f ? (m + log2f(lsum)) * kLn2 : -INFINITY;
   }
 
   tc_fence_before();
@@ -558,8 +641,12 @@ bool encode_map(CUtensorMap* m, const void* base, int D, long long rows, int hea
 }
 
 template <int D>
-cudaError_t launch_tc_typed(const TcParams& prm, int grid, cudaStream_t st) {
+cudaError_t launch_tc_typed(const TcParams& prm, int rows, cudaStream_t st) {
   const int smem = Cfg<D>::SMEM;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = rows < sms ? rows : sms;   // persistent: one CTA per SM
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -594,9 +681,10 @@ cudaError_t launch_attention_tc(const psa_params_t& p, const Layout& L, float sc
   prm.err = (int*)(ws + L.err);
   prm.Hq = p.Hq; prm.Hkv = p.Hkv; prm.N = p.N; prm.Nq = L.Nq; prm.Nk = L.Nk;
   prm.causal = p.causal;
+  prm.n_rows = BHq * L.Nq;
   prm.scale_log2 = scale * kLog2e;
-  const int grid = BHq * L.Nq;
-  return p.d == 128 ? launch_tc_typed<128>(prm, grid, st) : launch_tc_typed<64>(prm, grid, st);
+  return p.d == 128 ? launch_tc_typed<128>(prm, prm.n_rows, st)
+                    : launch_tc_typed<64>(prm, prm.n_rows, st);
 }
 
 }  // namespace psa

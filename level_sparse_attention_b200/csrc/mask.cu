@@ -15,9 +15,9 @@
 //
 // Three launches:
 //   qmean_kernel   one CTA per query block; streams Q once (HBM-bound).
-//   score_kernel   lanes = 32 query blocks of one head, warps walk KV blocks;
-//                  every lane reads the same level-3 key row (a broadcast load)
-//                  and keeps its q_bar in registers: 4 FMA per 16-byte load.
+//   score_kernel   lanes = 32 query blocks of one head, q_bar in registers;
+//                  chunks of level-3 keys staged in shared memory, read as
+//                  broadcast 16-byte loads, 8 independent FMA chains per lane.
 //   assign_kernel  one CTA per query block: softmax, bitonic sort of packed
 //                  (P, index) keys in shared memory, scan, cut, overrides, and
 //                  the work list (KV block indices grouped by level).
@@ -78,11 +78,32 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
 
 // -------------------------------------------------------------- scoring
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kScoreChunk = 8;       // KV blocks staged per step (one per warp)
+
+// Lanes = 32 query blocks of one head (q_bar in registers); the CTA walks a
+// range of KV blocks in chunks of 8, staging the chunk's 64 level-3 keys in
+// shared memory (cp.async, double-buffered).  Warp w scores KV block w of the
+// chunk: its 8 keys are read as broadcast 16-byte shared loads, 8 independent
+// FMA chains per lane.
 template <int D>
 __global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int splits,
                                                     const float* __restrict__ qmean,
                                                     const float* __restrict__ k3f,
                                                     float* __restrict__ zlog) {
+  extern __shared__ __align__(16) float ks[];        // [2][kScoreChunk * 8][D]
+  constexpr int KEYS = kScoreChunk * 8;
   const int groups = (a.Nq + 31) / 32;
   int id = blockIdx.x;
   const int split = id % splits; id /= splits;
@@ -105,36 +126,59 @@ __global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int splits,
   const float* kbase = k3f + (long long)bhk * rows3 * D;
   const int per = (a.Nk + splits - 1) / splits;
   const int j0 = split * per, j1 = min(a.Nk, j0 + per);
-  const int g_per_blk = a.kv_blk / 8;          // level-3 keys per KV block
-  for (int j = j0 + warp; j < j1; j += 8) {
-    const int g0 = j * g_per_blk;
-    const int ng = (int)min((long long)g_per_blk, rows3 - g0);
-    float mx = -INFINITY;
-    float lg[8];
+  const int n_chunks = j1 > j0 ? (j1 - j0 + kScoreChunk - 1) / kScoreChunk : 0;
+
+  auto stage = [&](int ci, int buf) {
+    const long long g0 = (long long)(j0 + ci * kScoreChunk) * 8;
+    float* dst = ks + (size_t)buf * KEYS * D;
+    for (int i = threadIdx.x; i < KEYS * D / 4; i += blockDim.x) {
+      const int key = i / (D / 4), c4 = i % (D / 4);
+      if (g0 + key < rows3) cp_async16(dst + key * D + c4 * 4, kbase + (g0 + key) * D + c4 * 4);
+    }
+    cp_async_commit();
+  };
+  if (n_chunks > 0) stage(0, 0);
+  for (int ci = 0; ci < n_chunks; ++ci) {
+    if (ci + 1 < n_chunks) {
+      stage(ci + 1, (ci + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int j = j0 + ci * kScoreChunk + warp;
+    if (j < j1) {
+      const float* kb = ks + (size_t)(ci & 1) * KEYS * D + warp * 8 * D;
+      const long long g0 = (long long)j * 8;
+      const int ng = (int)min(8LL, rows3 - g0);
+      float acc[8];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      lg[g] = -INFINITY;
-      if (g < ng) {
-        const float* k = kbase + (long long)(g0 + g) * D;
-        float acc = 0.f;
+      for (int g = 0; g < 8; ++g) acc[g] = 0.f;
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(k + c));
-          acc = fmaf(q[c], v.x, acc);
-          acc = fmaf(q[c + 1], v.y, acc);
-          acc = fmaf(q[c + 2], v.z, acc);
-          acc = fmaf(q[c + 3], v.w, acc);
+      for (int c = 0; c < D; c += 4) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 v = *reinterpret_cast<const float4*>(kb + g * D + c);
+          acc[g] = fmaf(q[c], v.x, acc[g]);
+          acc[g] = fmaf(q[c + 1], v.y, acc[g]);
+          acc[g] = fmaf(q[c + 2], v.z, acc[g]);
+          acc[g] = fmaf(q[c + 3], v.w, acc[g]);
         }
-        const int cnt = min(8, a.N - (g0 + g) * 8);
-        lg[g] = a.scale * acc + logf((float)cnt);
+      }
+      float lg[8], mx = -INFINITY;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int cnt = min(8, a.N - (int)(g0 + g) * 8);
+        lg[g] = g < ng ? a.scale * acc[g] + logf((float)cnt) : -INFINITY;
         mx = fmaxf(mx, lg[g]);
       }
-    }
-    float s = 0.f;
+      float s = 0.f;
 #pragma unroll
-    for (int g = 0; g < 8; ++g)
-      if (g < ng) s += expf(lg[g] - mx);
-    if (active) zlog[((long long)bhq * a.Nq + qa) * a.Nk + j] = mx + logf(s);
+      for (int g = 0; g < 8; ++g)
+        if (g < ng) s += expf(lg[g] - mx);
+      if (active) zlog[((long long)bhq * a.Nq + qa) * a.Nk + j] = mx + logf(s);
+    }
+    __syncthreads();
   }
 }
 
@@ -367,10 +411,17 @@ cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, ch
   const float* qm = (const float*)(ws + L.qmean);
   const float* k3 = (const float*)(ws + L.k3f);
   float* z = (float*)(ws + L.zlog);
-  if (p.d == 128)
-    score_kernel<128><<<grid, 256, 0, st>>>(a, splits, qm, k3, z);
-  else
-    score_kernel<64><<<grid, 256, 0, st>>>(a, splits, qm, k3, z);
+  const size_t smem = (size_t)2 * kScoreChunk * 8 * p.d * sizeof(float);
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    score_kernel<128><<<grid, 256, smem, st>>>(a, splits, qm, k3, z);
+  } else {
+    e = cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    score_kernel<64><<<grid, 256, smem, st>>>(a, splits, qm, k3, z);
+  }
   return cudaGetLastError();
 }
 
