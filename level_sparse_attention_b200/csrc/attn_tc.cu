@@ -12,17 +12,19 @@
 // Each pooled key's logit gets + log2(c) (c = tokens it averages) so that it
 // carries their softmax mass.
 //
-// CTA = one (batch, query head, 128-row query block), 6 warps:
+// Persistent CTAs (one per SM) walk the query blocks; per query block, 10 warps:
 //   warp 0     TMA producer: Q once; per tile, one 2-D box per sub-block and
 //              64-column half for K and for V (the box height is the level's
 //              sub-block height), plus a per-key bias / position table.
 //   warp 1     TMEM allocator and single-thread tcgen05.mma issuer:
 //              S[t%2] = Q K_t^T (SS form), then O += P_t V_t with P read from
 //              TMEM (TS form); commits signal the softmax and free stages.
-//   warps 2-5  softmax: one query row per thread (TMEM lane = row), online
-//              softmax in log2 units, P written back to TMEM as bf16, lazy O
+//   warps 2-9  softmax, two warpgroups: each row is shared by one thread of
+//              each group (TMEM lane = row), which take 64 keys of the tile
+//              each; online softmax in log2 units with the partial row maxima
+//              exchanged per tile, P written back to TMEM as bf16, lazy O
 //              rescale (only when the running max grows by more than 2^8),
-//              epilogue O / lse.
+//              epilogue O / lse split by column halves.
 // TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,384+d).
 // Every mbarrier wait is bounded: on expiry the kernel records a timeout in
 // the workspace error word and winds down without trapping.
@@ -36,11 +38,12 @@ namespace {
 
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per packed tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;     // producer, MMA, 2 softmax warpgroups
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
+constexpr int kListCache = 1024;         // work-list entries staged in shared memory
 
 template <int D>
 struct Cfg {
@@ -55,8 +58,11 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
   static constexpr int OFF_META = OFF_V + VSTAGES * KV_BYTES;   // per table: bias[128], kpos[128]
-  static constexpr int OFF_BAR = OFF_META + MSTAGES * 1024;
-  static constexpr int SMEM = OFF_BAR + 512 + 1024;             // + slack for 1024 alignment
+  static constexpr int META_BYTES = 128 + 1024;                // chunk biases, flag, per-key tables
+  static constexpr int OFF_BAR = OFF_META + MSTAGES * META_BYTES;
+  static constexpr int OFF_XCH = OFF_BAR + 512;                 // softmax pair exchange [2][2][128]
+  static constexpr int OFF_LIST = OFF_XCH + 2048;               // the query block's work list
+  static constexpr int SMEM = OFF_LIST + kListCache * 4 + 1024; // + slack for 1024 alignment
 };
 
 struct __align__(64) TcParams {
@@ -87,14 +93,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// One test of phase `parity`; a thread whose phase is not complete is
+// suspended until it completes or for at most ~1 ms, so that waiting warps do
+// not take issue slots from the warps they share a scheduler with.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -136,6 +145,59 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 instructions) and the exp2 polynomial
+
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair x <= 0 on the FMA pipes, so that only part of a tile's
+// exponentials queue on the transcendental unit.  Cody-Waite style: x is
+// clamped to >= -126, split as n + f with n = round(x) (the 1.5 * 2^23
+// addition rounds to an integer held in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f is a degree-3 polynomial whose coefficients were fitted
+// here for the least maximum relative error on that interval (7.5e-5, far
+// below the bf16 rounding of P); 2^n is added into the exponent field.
+// Inputs of -inf give 2^-126 rather than 0, so a row counts as holding keys
+// only once its running maximum is finite.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111400127411f, c3 = 0.0551716685295105f;
+  const uint64_t X = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t T = fadd2(X, f2pack(kMagic, kMagic));
+  const uint64_t N = fadd2(T, f2pack(-kMagic, -kMagic));
+  const uint64_t F = ffma2(N, f2pack(-1.f, -1.f), X);
+  uint64_t P = ffma2(F, f2pack(c3, c3), f2pack(c2, c2));
+  P = ffma2(P, F, f2pack(c1, c1));
+  P = ffma2(P, F, f2pack(c0, c0));
+  float p0, p1, t0, t1;
+  f2unpack(P, p0, p1);
+  f2unpack(T, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -224,44 +286,55 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 // ------------------------------------------------------------ work list
 
+// Per query block: entry counts per level give where each level starts in
+// the entry list (f1..f4) and in the packed key sequence (b1..b4).  Kept in
+// scalars (no arrays) so that lookups by a run-time level stay in registers.
 struct RowWork {
-  int first[kLevels + 1];   // entry index where level l starts (first[4] = entries)
-  int base[kLevels + 1];    // packed key offset where level l starts (base[4] = keys)
+  int f1, f2, f3, f4;       // first entry of level 1, 2, 3; number of entries
+  int b1, b2, b3, b4;       // first packed key of level 1, 2, 3; number of keys
   int tiles;
 };
 
 __device__ __forceinline__ RowWork row_work(int4 c) {
   RowWork w;
-  const int n[kLevels] = {c.x, c.y, c.z, c.w};
-  w.first[0] = 0;
-  w.base[0] = 0;
-  for (int l = 0; l < kLevels; ++l) {
-    w.first[l + 1] = w.first[l] + n[l];
-    w.base[l + 1] = w.base[l] + n[l] * (64 >> l);
-  }
-  w.tiles = (w.base[kLevels] + kBN - 1) / kBN;
+  w.f1 = c.x;
+  w.f2 = w.f1 + c.y;
+  w.f3 = w.f2 + c.z;
+  w.f4 = w.f3 + c.w;
+  w.b1 = 64 * c.x;
+  w.b2 = w.b1 + 32 * c.y;
+  w.b3 = w.b2 + 16 * c.z;
+  w.b4 = w.b3 + 8 * c.w;
+  w.tiles = (w.b4 + kBN - 1) / kBN;
   return w;
 }
 
-// The entries of tile t, one per lane: lane i takes entry e0 + i.  Entries
-// never cross a tile edge, so the lanes inside the tile form a prefix.
+__device__ __forceinline__ int sel4(int l, int a0, int a1, int a2, int a3) {
+  return l == 0 ? a0 : (l == 1 ? a1 : (l == 2 ? a2 : a3));
+}
+
+// The entries of tile t, one per lane: lane i takes the tile's first entry + i.
+// Entries never cross a tile edge, so the lanes inside the tile form a prefix.
 struct TileEntry {
   bool in_tile;
   int j, l, R, r0;          // KV block, level, sub-block rows, first row in the tile
 };
 
-__device__ __forceinline__ TileEntry tile_entry(const RowWork& w, const int* lrow, int e0, int t,
-                                                int lane) {
+__device__ __forceinline__ TileEntry tile_entry(const RowWork& w, const int* lrow,
+                                                const int* lcache, int t, int lane) {
+  // first entry of tile t: packed offset 128*t is always an entry boundary
+  const int off0 = t * kBN;
+  const int l0 = (off0 >= w.b1) + (off0 >= w.b2) + (off0 >= w.b3);
+  const int e = sel4(l0, 0, w.f1, w.f2, w.f3) + ((off0 - sel4(l0, 0, w.b1, w.b2, w.b3)) >> (6 - l0)) +
+                lane;
   TileEntry te;
-  const int e = e0 + lane;
-  int l = 0;
-  while (l < kLevels - 1 && e >= w.first[l + 1]) ++l;
+  const int l = (e >= w.f1) + (e >= w.f2) + (e >= w.f3);
   te.l = l;
   te.R = 64 >> l;
-  const int off = w.base[l] + (e - w.first[l]) * te.R;
-  te.in_tile = e < w.first[kLevels] && off < (t + 1) * kBN;
+  const int off = sel4(l, 0, w.b1, w.b2, w.b3) + ((e - sel4(l, 0, w.f1, w.f2, w.f3)) << (6 - l));
+  te.in_tile = e < w.f4 && off < (t + 1) * kBN;
   te.r0 = off - t * kBN;
-  te.j = te.in_tile ? __ldg(lrow + e) : 0;
+  te.j = te.in_tile ? (e < kListCache ? lcache[e] : __ldg(lrow + e)) : 0;
   return te;
 }
 
@@ -297,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     mbar_init(bar(B_QEMPTY), 1);
     for (int s = 0; s < KS; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
-    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 1); mbar_init(bar(B_MEMPTY + s), 4); }
+    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 8); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PFULL + i), 128);
+      mbar_init(bar(B_PFULL + i), 256);
       mbar_init(bar(B_ODONE + i), 1);
     }
     mbar_init(bar(B_FINAL), 1);
@@ -339,6 +412,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int bhk = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / (p.Hq / p.Hkv);
       const int* lrow = p.list + (long long)item * p.Nk;
+      // stage the work list (first kListCache entries) once per query block
+      int* lcache = reinterpret_cast<int*>(smem + C::OFF_LIST);
+      const int n_ent = min(w.f4, kListCache);
+      __syncwarp();
+      for (int i = lane; i < n_ent; i += 32) lcache[i] = __ldg(lrow + i);
+      __syncwarp();
+      TileEntry cur = tile_entry(w, lrow, lcache, 0, lane), prev = cur;
       if (iq > 0 && !warp_wait(bar(B_QEMPTY), (iq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
       if (lane == 0) {
         mbar_expect_tx(bar(B_QFULL), C::Q_BYTES);
@@ -347,76 +427,89 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                       qa * kBM, bhq);
       }
       ++iq;
-      int ek = 0, ev = 0;
       for (int t = 0; t <= T; ++t) {
+        // the next tile's list entries are loaded before this tile's waits
+        const TileEntry nxt = t + 1 < T ? tile_entry(w, lrow, lcache, t + 1, lane) : cur;
         if (t < T) {
           // K of tile t, and its per-key bias / position table
           const int s = gk % KS, ms = gk % MS;
           if (gk >= KS && !warp_wait(bar(B_KEMPTY + s), ((gk / KS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
           if (gk >= MS && !warp_wait(bar(B_MEMPTY + ms), ((gk / MS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          const TileEntry te = tile_entry(w, lrow, ek, t, lane);
-          const unsigned ballot = __ballot_sync(0xffffffffu, te.in_tile);
-          const int n_in = __popc(ballot);
-          int bytes = te.in_tile ? te.R * D * 2 : 0;
+          const int n_in = __popc(__ballot_sync(0xffffffffu, cur.in_tile));
+          int bytes = cur.in_tile ? cur.R * D * 2 : 0;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-          // table: lane covers columns 4*lane .. 4*lane+3 (inside one 8-column chunk)
-          const int col = 4 * lane;
+          // Per-key bias table of this tile.  Usually every key of an 8-key
+          // chunk has bias = its level (log2 of the pool factor), so 16 chunk
+          // values describe the tile.  Tiles holding the ragged last KV block
+          // (partial groups, rows past the end) or, causally, a block that
+          // straddles the diagonal (token positions) get a full per-key table.
+          unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
+          float* cbias = reinterpret_cast<float*>(mt_base);                 // [16]
+          int* mflag = reinterpret_cast<int*>(mt_base + 64);
+          float* mbias = reinterpret_cast<float*>(mt_base + 128);           // [128]
+          int* mpos = reinterpret_cast<int*>(mt_base + 128 + 512);          // [128]
+          const bool special = cur.in_tile && (cur.j == p.Nk - 1 ||
+                               (p.causal && cur.l == 0 &&
+                                (cur.j + 1) * 64 - 1 >= qa * kBM));
+          const bool slow = __any_sync(0xffffffffu, special);
+          const int col = slow ? 4 * lane : 8 * (lane & 15);
           int owner = 0;
           for (int i = 1; i < n_in; ++i)
-            if (__shfl_sync(0xffffffffu, te.r0, i) <= col) owner = i;
-          const int oj = __shfl_sync(0xffffffffu, te.j, owner);
-          const int ol = __shfl_sync(0xffffffffu, te.l, owner);
-          const int oR = __shfl_sync(0xffffffffu, te.R, owner);
-          const int or0 = __shfl_sync(0xffffffffu, te.r0, owner);
+            if (__shfl_sync(0xffffffffu, cur.r0, i) <= col) owner = i;
+          const int oj = __shfl_sync(0xffffffffu, cur.j, owner);
+          const int ol = __shfl_sync(0xffffffffu, cur.l, owner);
+          const int oR = __shfl_sync(0xffffffffu, cur.R, owner);
+          const int or0 = __shfl_sync(0xffffffffu, cur.r0, owner);
           const bool live = n_in > 0 && col < or0 + oR;   // false past the last entry
-          float bias[4];
-          int kpos[4];
+          if (!slow) {
+            if (lane < 16) cbias[lane] = live ? (float)ol : -INFINITY;
+            if (lane == 16) *mflag = 0;
+          } else {
+            float bias[4];
+            int kpos[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const long long g = (long long)oj * oR + (col + c - or0);
-            const long long tok = g << ol;
-            const int cnt = (int)min((long long)(1 << ol), (long long)p.N - tok);
-            bias[c] = !live || cnt <= 0 ? -INFINITY : (cnt == (1 << ol) ? (float)ol : log2f((float)cnt));
-            kpos[c] = (live && p.causal && ol == 0) ? (int)tok : INT_MIN;
+            for (int c = 0; c < 4; ++c) {
+              const int g = oj * oR + (col + c - or0);
+              const int tok = g << ol;
+              const int cnt = min(1 << ol, p.N - tok);
+              bias[c] = !live || cnt <= 0 ? -INFINITY : (cnt == (1 << ol) ? (float)ol : log2f((float)cnt));
+              kpos[c] = (live && p.causal && ol == 0) ? tok : INT_MIN;
+            }
+            reinterpret_cast<float4*>(mbias)[lane] = make_float4(bias[0], bias[1], bias[2], bias[3]);
+            reinterpret_cast<int4*>(mpos)[lane] = make_int4(kpos[0], kpos[1], kpos[2], kpos[3]);
+            if (lane == 0) *mflag = 1;
           }
-          float* mb = reinterpret_cast<float*>(smem + C::OFF_META + ms * 1024);
-          reinterpret_cast<float4*>(mb)[lane] = make_float4(bias[0], bias[1], bias[2], bias[3]);
-          reinterpret_cast<int4*>(mb + kBN)[lane] = make_int4(kpos[0], kpos[1], kpos[2], kpos[3]);
-          __threadfence_block();
+          mbar_arrive(bar(B_MFULL + ms));           // each lane releases its own table writes
+          if (lane == 0) mbar_expect_tx(bar(B_KFULL + s), bytes);
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(bar(B_MFULL + ms));
-            mbar_expect_tx(bar(B_KFULL + s), bytes);
-          }
-          __syncwarp();
-          if (te.in_tile) {
-            const uint32_t kdst = sbase + C::OFF_K + s * C::KV_BYTES + te.r0 * 128;
+          if (cur.in_tile) {
+            const uint32_t kdst = sbase + C::OFF_K + s * C::KV_BYTES + cur.r0 * 128;
             for (int h = 0; h < C::HALVES; ++h)
-              tma_load_3d(kdst + h * C::HALF, &p.tk[te.l], bar(B_KFULL + s), h * 64, te.j * te.R, bhk);
+              tma_load_3d(kdst + h * C::HALF, &p.tk[cur.l], bar(B_KFULL + s), h * 64,
+                          cur.j * cur.R, bhk);
           }
-          ek += n_in;
           ++gk;
         }
         if (t >= 1) {
-          // V of tile t - 1
+          // V of tile t - 1 (same entries as its K)
           const int s = gv % VS;
           if (gv >= VS && !warp_wait(bar(B_VEMPTY + s), ((gv / VS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          const TileEntry te = tile_entry(w, lrow, ev, t - 1, lane);
-          const int n_in = __popc(__ballot_sync(0xffffffffu, te.in_tile));
-          int bytes = te.in_tile ? te.R * D * 2 : 0;
+          int bytes = prev.in_tile ? prev.R * D * 2 : 0;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
           if (lane == 0) mbar_expect_tx(bar(B_VFULL + s), bytes);
           __syncwarp();
-          if (te.in_tile) {
-            const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + te.r0 * 128;
+          if (prev.in_tile) {
+            const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + prev.r0 * 128;
             for (int h = 0; h < C::HALVES; ++h)
-              tma_load_3d(vdst + h * C::HALF, &p.tv[te.l], bar(B_VFULL + s), h * 64, te.j * te.R, bhk);
+              tma_load_3d(vdst + h * C::HALF, &p.tv[prev.l], bar(B_VFULL + s), h * 64,
+                          prev.j * prev.R, bhk);
           }
-          ev += n_in;
           ++gv;
         }
+        prev = cur;
+        cur = nxt;
       }
     }
   } else if (warp == 1) {
@@ -474,9 +567,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else {
     // --------------------------------------------------------------- softmax
+    // Two warpgroups share every row: group hg takes keys [64*hg, 64*hg + 64)
+    // of each tile and O columns [hg*D/2, (hg+1)*D/2).  The pair of warps that
+    // own the same 32 rows (same TMEM lane quadrant) exchange their partial
+    // row maxima every tile through shared memory and a 64-thread named
+    // barrier, so both keep the same running max; the partial row sums are
+    // added at the end.  Both warps of a pair always take the same number of
+    // barriers, also when a wait has timed out, so the barrier cannot hang.
+    constexpr int HD = D / 2;
+    constexpr int NPOLY = 24;      // columns of each 64 whose 2^x runs on the FMA pipes
+    const int hg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][2][128]
+    int nx = 0;                                                 // exchanges so far
+    auto exchange = [&](float v) -> float {   // returns the partner's value
+      float* buf = xch + (nx & 1) * 256;
+      buf[hg * 128 + r] = v;
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+      ++nx;
+      return buf[(1 - hg) * 128 + r];
+    };
+    const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
     int g = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -484,97 +597,143 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int qpos = qa * kBM + r;
       float m = -INFINITY, lsum = 0.f;
-      for (int t = 0; ok && t < T; ++t) {
+      for (int t = 0; t < T; ++t) {
         const int gt = g + t, bb = gt & 1, ms = gt % MS;
-        if (!warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) ||
-            !warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float* mbias = reinterpret_cast<const float*>(smem + C::OFF_META + ms * 1024);
-        const int* mpos = reinterpret_cast<const int*>(mbias + kBN);
-        float x[kBN];
-#pragma unroll
-        for (int c0 = 0; c0 < kBN; c0 += 32)
-          tmem_ld32(T_S + bb * 128 + lane_off + c0, reinterpret_cast<uint32_t*>(x + c0));
-        tmem_ld_wait();
-        reg_fence<kBN>(reinterpret_cast<uint32_t*>(x));
+        ok = ok && warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) &&
+             warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err);
+        float x[64];
         float mt = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+          const unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
+          const bool slow = *reinterpret_cast<const int*>(mt_base + 64) != 0;
+          const float* cb = reinterpret_cast<const float*>(mt_base) + 8 * hg;
+          const float* mbias = reinterpret_cast<const float*>(mt_base + 128) + 64 * hg;
+          const int* mpos = reinterpret_cast<const int*>(mt_base + 128 + 512) + 64 * hg;
+          const float4 cb0 = *reinterpret_cast<const float4*>(cb);
+          const float4 cb1 = *reinterpret_cast<const float4*>(cb + 4);
+          const float cbv[8] = {cb0.x, cb0.y, cb0.z, cb0.w, cb1.x, cb1.y, cb1.z, cb1.w};
+          const uint32_t sa = T_S + bb * 128 + lane_off + 64 * hg;
+          tmem_ld32(sa, reinterpret_cast<uint32_t*>(x));
+          tmem_ld_wait();
+          reg_fence<32>(reinterpret_cast<uint32_t*>(x));
+          tmem_ld32(sa + 32, reinterpret_cast<uint32_t*>(x + 32));   // in flight during the first half
+          float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kBN; c += 4) {
-          const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
-          x[c] = fmaf(x[c], p.scale_log2, b4.x);
-          x[c + 1] = fmaf(x[c + 1], p.scale_log2, b4.y);
-          x[c + 2] = fmaf(x[c + 2], p.scale_log2, b4.z);
-          x[c + 3] = fmaf(x[c + 3], p.scale_log2, b4.w);
-          if (p.causal) {
-            const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
-            if (qpos < k4.x) x[c] = -INFINITY;
-            if (qpos < k4.y) x[c + 1] = -INFINITY;
-            if (qpos < k4.z) x[c + 2] = -INFINITY;
-            if (qpos < k4.w) x[c + 3] = -INFINITY;
+          for (int half = 0; half < 2; ++half) {
+            if (half == 1) {
+              tmem_ld_wait();
+              reg_fence<32>(reinterpret_cast<uint32_t*>(x + 32));
+            }
+            if (!slow) {
+#pragma unroll
+              for (int c = half * 32; c < half * 32 + 32; c += 4) {
+                const float b = cbv[c >> 3];
+                const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b, b));
+                const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b, b));
+                f2unpack(v01, x[c], x[c + 1]);
+                f2unpack(v23, x[c + 2], x[c + 3]);
+                mx0 = fmax3(mx0, x[c], x[c + 1]);
+                mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int c = half * 32; c < half * 32 + 32; c += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
+                const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b4.x, b4.y));
+                const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b4.z, b4.w));
+                f2unpack(v01, x[c], x[c + 1]);
+                f2unpack(v23, x[c + 2], x[c + 3]);
+                if (p.causal) {
+                  const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
+                  if (qpos < k4.x) x[c] = -INFINITY;
+                  if (qpos < k4.y) x[c + 1] = -INFINITY;
+                  if (qpos < k4.z) x[c + 2] = -INFINITY;
+                  if (qpos < k4.w) x[c + 3] = -INFINITY;
+                }
+                mx0 = fmax3(mx0, x[c], x[c + 1]);
+                mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+              }
+            }
           }
-          mt = fmaxf(mt, fmaxf(fmaxf(x[c], x[c + 1]), fmaxf(x[c + 2], x[c + 3])));
+          mt = fmaxf(mx0, mx1);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
+        const float other = exchange(mt);
+        if (!ok) continue;
+        mt = hg == 0 ? fmaxf(mt, other) : fmaxf(other, mt);
         const float m_new = fmaxf(m, mt);
         const bool need = m_new > m + kRescaleLog2;     // false while both are -inf
         if (__any_sync(0xffffffffu, need)) {
           const float m_use = need ? m_new : m;
           const float factor = need ? ex2(m - m_use) : 1.f;   // 0 when m = -inf
           if (t > 0) {
-            if (!warp_wait(bar(B_ODONE + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, abort_flag, p.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+            ok = warp_wait(bar(B_ODONE + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, abort_flag, p.err);
+            if (ok) {
+              tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(T_O + lane_off + c0, o);
-              tmem_ld_wait();
-              reg_fence<32>(o);
+              for (int c0 = 0; c0 < HD; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(T_O + lane_off + hg * HD + c0, o);
+                tmem_ld_wait();
+                reg_fence<32>(o);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-              tmem_st32(T_O + lane_off + c0, o);
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+                tmem_st32(T_O + lane_off + hg * HD + c0, o);
+              }
             }
           }
           lsum *= factor;
           m = m_use;
         }
+        if (!ok) continue;
         const float m_base = m == -INFINITY ? 0.f : m;
+        const uint64_t nm2 = f2pack(-m_base, -m_base);
+        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+        uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2(x[h * 64 + c] - m_base);
-            const float p1 = ex2(x[h * 64 + c + 1] - m_base);
-            lsum += p0 + p1;
-            __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
-            pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
+        for (int c = 0; c < 64; c += 2) {
+          float p0, p1;
+          const uint64_t d = fadd2(f2pack(x[c], x[c + 1]), nm2);
+          float d0, d1;
+          f2unpack(d, d0, d1);
+          if (c < NPOLY) {
+            exp2_poly2(d0, d1, p0, p1);
+          } else {
+            p0 = ex2(d0);
+            p1 = ex2(d1);
           }
-          tmem_st32(T_P + bb * 64 + lane_off + h * 32, pk);
+          if ((c >> 1) & 1) acc1 = fadd2(acc1, f2pack(p0, p1));
+          else acc0 = fadd2(acc0, f2pack(p0, p1));
+          __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+          pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
         }
+        tmem_st32(T_P + bb * 64 + lane_off + 32 * hg, pk);
+        float a0, a1, a2, a3;
+        f2unpack(acc0, a0, a1);
+        f2unpack(acc1, a2, a3);
+        lsum += (a0 + a1) + (a2 + a3);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL + bb));
       }
-      // epilogue of this query block
+      // epilogue of this query block: full row sum, then this group's O columns
+      const float other = exchange(lsum);
+      const float ltot = hg == 0 ? lsum + other : other + lsum;
       const bool row_ok = qpos < p.N;
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D;
+      const bool keys = m > -INFINITY;                  // the row kept at least one key
+      const float inv = keys ? 1.f / ltot : 0.f;
+      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D + hg * HD;
       const bool have_o = __all_sync(0xffffffffu, ok) && T > 0 &&
                           warp_wait(bar(B_ODONE + ((g + T - 1) & 1)), ((g + T - 1) >> 1) & 1,
                                     abort_flag, p.err);
       if (have_o) tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < HD; c0 += 32) {
         uint32_t o[32];
         if (have_o) {
-          tmem_ld32(T_O + lane_off + c0, o);
+          tmem_ld32(T_O + lane_off + hg * HD + c0, o);
           tmem_ld_wait();
           reg_fence<32>(o);
         } else {
@@ -595,10 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (row_ok && p.lse)
-        p.lse[(long long)bhq * p.N + qpos] = lsum > 0.f ? (m + log2f(lsum)) * kLn2 : -INFINITY;
+      if (row_ok && p.lse && hg == 0)
+        p.lse[(long long)bhq * p.N + qpos] = keys ? (m + log2f(ltot)) * kLn2 : -INFINITY;
       g += T;
-      if (!ok) break;
     }
   }
 
