@@ -15,10 +15,10 @@
 //
 // Three launches:
 //   qmean_kernel   one CTA per query block; streams Q once (HBM-bound).
-//   score_kernel   lanes = 32 query blocks of one head, q_bar in registers;
-//                  chunks of level-3 keys staged in shared memory, read as
-//                  broadcast 16-byte loads, 8 independent FMA chains per lane.
-//   assign_kernel  one CTA per query block: softmax, bitonic sort of packed
+//   score_kernel   register-tiled fp32 GEMM of query-block means against the
+//                  level-3 keys, logsumexp over each KV block's keys fused
+//                  into the epilogue.
+//   assign_kernel  one warp per query block: softmax, bitonic sort of packed
 //                  (P, index) keys in shared memory, scan, cut, overrides, and
 //                  the work list (KV block indices grouped by level).
 #include "psa_internal.cuh"
@@ -78,206 +78,183 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
 
 // -------------------------------------------------------------- scoring
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+constexpr int kSgM = 64;       // query blocks per CTA tile
+constexpr int kSgN = 128;      // level-3 keys per CTA tile (16 KV blocks of 8 keys)
+constexpr int kSgK = 16;       // head-dim slice per stage
+constexpr int kSgPad = 4;      // row padding of the transposed shared tiles
 
-constexpr int kScoreChunk = 8;       // KV blocks staged per step (one per warp)
-
-// Lanes = 32 query blocks of one head (q_bar in registers); the CTA walks a
-// range of KV blocks in chunks of 8, staging the chunk's 64 level-3 keys in
-// shared memory (cp.async, double-buffered).  Warp w scores KV block w of the
-// chunk: its 8 keys are read as broadcast 16-byte shared loads, 8 independent
-// FMA chains per lane.
+// Block logits as a register-tiled fp32 GEMM, C = q_bar [Nq x d] . K3 [rows3 x d]^T
+// per head, with the logsumexp over each KV block's 8 level-3 keys fused into
+// the epilogue.  256 threads; thread (tm, tn) owns 4 query blocks x the 8 keys
+// of one KV block, so its 32 accumulators give 4 block logits directly.
+// Operands are staged transposed in shared memory ([k][m], [k][n]),
+// double-buffered through registers: per k-step a thread reads 3 x 16 bytes
+// and issues 32 FMA.
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int splits,
+__global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int m_tiles, int n_tiles,
                                                     const float* __restrict__ qmean,
                                                     const float* __restrict__ k3f,
                                                     float* __restrict__ zlog) {
-  extern __shared__ __align__(16) float ks[];        // [2][kScoreChunk * 8][D]
-  constexpr int KEYS = kScoreChunk * 8;
-  const int groups = (a.Nq + 31) / 32;
+  __shared__ __align__(16) float As[2][kSgK][kSgM + kSgPad];
+  __shared__ __align__(16) float Bs[2][kSgK][kSgN + kSgPad];
   int id = blockIdx.x;
-  const int split = id % splits; id /= splits;
-  const int grp = id % groups;
-  const int bhq = id / groups;
+  const int nt = id % n_tiles; id /= n_tiles;
+  const int mt = id % m_tiles;
+  const int bhq = id / m_tiles;
   const int b = bhq / a.Hq, hq = bhq % a.Hq;
   const int bhk = b * a.Hkv + hq / (a.Hq / a.Hkv);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int qa = grp * 32 + lane;
-  const bool active = qa < a.Nq;
-
-  float q[D];
-  const float* qsrc = qmean + ((long long)bhq * a.Nq + (active ? qa : 0)) * D;
-#pragma unroll
-  for (int c = 0; c < D; c += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(qsrc + c);
-    q[c] = v.x; q[c + 1] = v.y; q[c + 2] = v.z; q[c + 3] = v.w;
-  }
   const long long rows3 = ((long long)a.N + 7) / 8;
-  const float* kbase = k3f + (long long)bhk * rows3 * D;
-  const int per = (a.Nk + splits - 1) / splits;
-  const int j0 = split * per, j1 = min(a.Nk, j0 + per);
-  const int n_chunks = j1 > j0 ? (j1 - j0 + kScoreChunk - 1) / kScoreChunk : 0;
+  const int m0 = mt * kSgM;
+  const long long n0 = (long long)nt * kSgN;
+  const float* Ag = qmean + (long long)bhq * a.Nq * D;
+  const float* Bg = k3f + (long long)bhk * rows3 * D;
+  const int tid = threadIdx.x;
+  const int tm = tid >> 4, tn = tid & 15;
 
-  auto stage = [&](int ci, int buf) {
-    const long long g0 = (long long)(j0 + ci * kScoreChunk) * 8;
-    float* dst = ks + (size_t)buf * KEYS * D;
-    for (int i = threadIdx.x; i < KEYS * D / 4; i += blockDim.x) {
-      const int key = i / (D / 4), c4 = i % (D / 4);
-      if (g0 + key < rows3) cp_async16(dst + key * D + c4 * 4, kbase + (g0 + key) * D + c4 * 4);
-    }
-    cp_async_commit();
+  // global -> register staging: A 64x16 (one float4 per thread), B 128x16 (two)
+  const int ar = tid >> 2, ak = (tid & 3) * 4;
+  const int br0 = tid >> 2, br1 = br0 + 64, bk = (tid & 3) * 4;
+  float4 ra, rb0, rb1;
+  auto load = [&](int k0) {
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    ra = (m0 + ar < a.Nq) ? *reinterpret_cast<const float4*>(Ag + (long long)(m0 + ar) * D + k0 + ak) : zero;
+    rb0 = (n0 + br0 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br0) * D + k0 + bk)) : zero;
+    rb1 = (n0 + br1 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br1) * D + k0 + bk)) : zero;
   };
-  if (n_chunks > 0) stage(0, 0);
-  for (int ci = 0; ci < n_chunks; ++ci) {
-    if (ci + 1 < n_chunks) {
-      stage(ci + 1, (ci + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  auto store = [&](int buf) {
+    As[buf][ak + 0][ar] = ra.x; As[buf][ak + 1][ar] = ra.y;
+    As[buf][ak + 2][ar] = ra.z; As[buf][ak + 3][ar] = ra.w;
+    Bs[buf][bk + 0][br0] = rb0.x; Bs[buf][bk + 1][br0] = rb0.y;
+    Bs[buf][bk + 2][br0] = rb0.z; Bs[buf][bk + 3][br0] = rb0.w;
+    Bs[buf][bk + 0][br1] = rb1.x; Bs[buf][bk + 1][br1] = rb1.y;
+    Bs[buf][bk + 2][br1] = rb1.z; Bs[buf][bk + 3][br1] = rb1.w;
+  };
+
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+
+  load(0);
+  store(0);
+  __syncthreads();
+  constexpr int NK = D / kSgK;
+#pragma unroll 1
+  for (int kt = 0; kt < NK; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < NK) load((kt + 1) * kSgK);
+#pragma unroll
+    for (int k = 0; k < kSgK; ++k) {
+      const float4 av = *reinterpret_cast<const float4*>(&As[buf][k][tm * 4]);
+      const float4 bv0 = *reinterpret_cast<const float4*>(&Bs[buf][k][tn * 8]);
+      const float4 bv1 = *reinterpret_cast<const float4*>(&Bs[buf][k][tn * 8 + 4]);
+      const float am[4] = {av.x, av.y, av.z, av.w};
+      const float bn[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(am[i], bn[c], acc[i][c]);
     }
-    __syncthreads();
-    const int j = j0 + ci * kScoreChunk + warp;
-    if (j < j1) {
-      const float* kb = ks + (size_t)(ci & 1) * KEYS * D + warp * 8 * D;
-      const long long g0 = (long long)j * 8;
-      const int ng = (int)min(8LL, rows3 - g0);
-      float acc[8];
-#pragma unroll
-      for (int g = 0; g < 8; ++g) acc[g] = 0.f;
-#pragma unroll
-      for (int c = 0; c < D; c += 4) {
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float4 v = *reinterpret_cast<const float4*>(kb + g * D + c);
-          acc[g] = fmaf(q[c], v.x, acc[g]);
-          acc[g] = fmaf(q[c + 1], v.y, acc[g]);
-          acc[g] = fmaf(q[c + 2], v.z, acc[g]);
-          acc[g] = fmaf(q[c + 3], v.w, acc[g]);
-        }
-      }
-      float lg[8], mx = -INFINITY;
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const int cnt = min(8, a.N - (int)(g0 + g) * 8);
-        lg[g] = g < ng ? a.scale * acc[g] + logf((float)cnt) : -INFINITY;
-        mx = fmaxf(mx, lg[g]);
-      }
-      float s = 0.f;
-#pragma unroll
-      for (int g = 0; g < 8; ++g)
-        if (g < ng) s += expf(lg[g] - mx);
-      if (active) zlog[((long long)bhq * a.Nq + qa) * a.Nk + j] = mx + logf(s);
+    if (kt + 1 < NK) {
+      store(buf ^ 1);
+      __syncthreads();
     }
-    __syncthreads();
+  }
+
+  // epilogue: block logit = logsumexp over the KV block's level-3 keys
+  const long long j = n0 / 8 + tn;
+  if (j >= a.Nk) return;
+  const long long g0 = j * 8;
+  float lnc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const long long g = g0 + c;
+    lnc[c] = g < rows3 ? logf((float)min(8LL, (long long)a.N - g * 8)) : -INFINITY;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int qa = m0 + tm * 4 + i;
+    if (qa >= a.Nq) continue;
+    float lg[8], mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      lg[c] = lnc[c] == -INFINITY ? -INFINITY : a.scale * acc[i][c] + lnc[c];
+      mx = fmaxf(mx, lg[c]);
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (lg[c] != -INFINITY) s += expf(lg[c] - mx);
+    zlog[((long long)bhq * a.Nq + qa) * a.Nk + j] = mx + logf(s);
   }
 }
 
 // ------------------------------------------------------------ assignment
+//
+// One warp per query block: no block-wide barriers.  The warp keeps its row's
+// packed (P, index) keys in shared memory and sorts them with a bitonic
+// network (lanes take strided compare-exchanges, __syncwarp between stages).
 
-__device__ __forceinline__ int block_sum_int(int v, int* red) {
-  // returns the exclusive prefix of v over threads and writes the total to red[32]
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    int t = lane < nw ? red[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
-    }
-    if (lane < nw) red[lane] = t - (lane < nw ? red[lane] : 0);   // exclusive warp offsets
-    if (lane == nw - 1) red[32] = t;
-  }
-  __syncthreads();
-  const int excl = red[warp] + x - v;
-  __syncthreads();
-  return excl;
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
-
-__device__ __forceinline__ float block_sum_float_excl(float v, float* red, float* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float x = v;
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+template <typename T>
+__device__ __forceinline__ T warp_excl_scan(T v, T* total) {
+  const int lane = threadIdx.x & 31;
+  T x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    const T y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    float t = lane < nw ? red[lane] : 0.f;
-    const float own = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
-    }
-    if (lane < nw) red[lane] = t - own;
-    if (lane == nw - 1) red[32] = t;
-  }
-  __syncthreads();
-  const float excl = red[warp] + (x - v);
-  if (total) *total = red[32];
-  __syncthreads();
-  return excl;
+  *total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
 }
 
 // Writes the work list of one query block from its level row `lev` (shared):
 // KV block indices at level 0, then 1, 2, 3, each in increasing index order.
-__device__ void emit_list(const int8_t* lev, int Nk, int* __restrict__ list_row,
-                          int4* __restrict__ count_row, int* red) {
-  const int per = (Nk + blockDim.x - 1) / blockDim.x;
-  const int j0 = threadIdx.x * per;
+__device__ void emit_list_warp(const int8_t* lev, int Nk, int* __restrict__ list_row,
+                               int4* __restrict__ count_row) {
+  const int lane = threadIdx.x & 31;
+  const int per = (Nk + 31) / 32;
+  const int j0 = lane * per, j1 = min(Nk, j0 + per);
   int base = 0;
   int cnt[kLevels];
+#pragma unroll
   for (int l = 0; l < kLevels; ++l) {
     int mine = 0;
-    for (int j = j0; j < min(Nk, j0 + per); ++j) mine += lev[j] == l;
-    const int excl = block_sum_int(mine, red);
-    const int total = red[32];
-    __syncthreads();
-    int pos = base + excl;
-    for (int j = j0; j < min(Nk, j0 + per); ++j)
+    for (int j = j0; j < j1; ++j) mine += lev[j] == l;
+    int total;
+    int pos = base + warp_excl_scan(mine, &total);
+    for (int j = j0; j < j1; ++j)
       if (lev[j] == l) list_row[pos++] = j;
     cnt[l] = total;
     base += total;
   }
-  if (threadIdx.x == 0) *count_row = make_int4(cnt[0], cnt[1], cnt[2], cnt[3]);
+  if (lane == 0) *count_row = make_int4(cnt[0], cnt[1], cnt[2], cnt[3]);
 }
 
-__global__ void __launch_bounds__(256) assign_kernel(MaskArgs a, int n2,
-                                                     const float* __restrict__ zlog,
-                                                     int8_t* __restrict__ map_ws,
-                                                     int8_t* __restrict__ map_user,
-                                                     float* __restrict__ mass_user,
-                                                     int* __restrict__ list,
-                                                     int4* __restrict__ counts) {
+__global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
+                              const float* __restrict__ zlog, int8_t* __restrict__ map_ws,
+                              int8_t* __restrict__ map_user, float* __restrict__ mass_user,
+                              int* __restrict__ list, int4* __restrict__ counts) {
   extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem);   // [n2]
-  int8_t* lev = reinterpret_cast<int8_t*>(key + n2);                          // [Nk]
-  __shared__ float redf[33];
-  __shared__ int redi[33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * rows_per_cta + warp;
+  if (row >= nrows) return;                 // whole warp; no block barriers below
+  const int lev_stride = (a.Nk + 15) & ~15;
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem) + (size_t)warp * n2;
+  int8_t* lev = reinterpret_cast<int8_t*>(smem + (size_t)rows_per_cta * n2 * 8) +
+                (size_t)warp * lev_stride;
 
-  const int row = blockIdx.x;
   const int qa = row % a.Nq;
   const int q_lo = qa * a.q_blk;
   const int q_hi = min(a.N, q_lo + a.q_blk) - 1;
@@ -286,98 +263,87 @@ __global__ void __launch_bounds__(256) assign_kernel(MaskArgs a, int n2,
 
   // softmax over the visible blocks
   float mx = -INFINITY;
-  for (int j = threadIdx.x; j < nvis; j += blockDim.x) mx = fmaxf(mx, z[j]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  mx = -INFINITY;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, redf[w]);
-  __syncthreads();
+  for (int j = lane; j < nvis; j += 32) mx = fmaxf(mx, z[j]);
+  mx = warp_max(mx);
   float part = 0.f;
-  for (int j = threadIdx.x; j < nvis; j += blockDim.x) part += expf(z[j] - mx);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = part;
-  __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += redf[w];
-  __syncthreads();
-  const float inv = 1.0f / tot;
+  for (int j = lane; j < nvis; j += 32) part += expf(z[j] - mx);
+  const float inv = 1.0f / warp_sum(part);
 
-  for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+  for (int i = lane; i < n2; i += 32) {
     unsigned long long k = 0ull;
     if (i < nvis) {
-      const float p = expf(z[i] - mx) * inv;
-      k = ((unsigned long long)__float_as_uint(p) << 32) | (0xffffffffu - (unsigned)i);
+      const float pj = expf(z[i] - mx) * inv;
+      k = ((unsigned long long)__float_as_uint(pj) << 32) | (0xffffffffu - (unsigned)i);
     }
     key[i] = k;
   }
-  for (int j = threadIdx.x; j < a.Nk; j += blockDim.x) lev[j] = -1;
-  __syncthreads();
+  for (int j = lane; j < a.Nk; j += 32) lev[j] = -1;
+  __syncwarp();
 
   // bitonic sort, descending: P high, then lower index first
   for (int k = 2; k <= n2; k <<= 1) {
-    for (int s = k >> 1; s > 0; s >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int ixj = i ^ s;
+    for (int sd = k >> 1; sd > 0; sd >>= 1) {
+      for (int i = lane; i < n2; i += 32) {
+        const int ixj = i ^ sd;
         if (ixj > i) {
           const unsigned long long u = key[i], v = key[ixj];
           const bool desc = (i & k) == 0;
           if (desc ? (u < v) : (u > v)) { key[i] = v; key[ixj] = u; }
         }
       }
-      __syncthreads();
+      __syncwarp();
     }
   }
 
-  // exclusive running mass in rank order, then the threshold cut
-  const int per = (n2 + blockDim.x - 1) / blockDim.x;
-  const int r0 = threadIdx.x * per;
+  // exclusive running mass in rank order (lanes take contiguous rank ranges)
+  const int per = (nvis + 31) / 32;
+  const int r0 = lane * per, r1 = min(nvis, r0 + per);
   float mine = 0.f;
-  for (int r = r0; r < min(nvis, r0 + per); ++r) mine += __uint_as_float((unsigned)(key[r] >> 32));
-  float c = block_sum_float_excl(mine, redf, nullptr);
-  for (int r = r0; r < min(nvis, r0 + per); ++r) {
-    const float p = __uint_as_float((unsigned)(key[r] >> 32));
+  for (int r = r0; r < r1; ++r) mine += __uint_as_float((unsigned)(key[r] >> 32));
+  float total;
+  float c = warp_excl_scan(mine, &total);
+  for (int r = r0; r < r1; ++r) {
+    const float pr = __uint_as_float((unsigned)(key[r] >> 32));
     const int j = (int)(0xffffffffu - (unsigned)(key[r] & 0xffffffffu));
     int l = -1;
 #pragma unroll
     for (int t = kLevels - 1; t >= 0; --t)
       if (c < a.tau[t]) l = t;
     lev[j] = (int8_t)l;
-    c += p;
+    c += pr;
   }
-  __syncthreads();
+  __syncwarp();
   // overrides: causal diagonal -> 0, forced prefix -> 0 (visible blocks only)
-  for (int j = threadIdx.x; j < nvis; j += blockDim.x) {
+  for (int j = lane; j < nvis; j += 32) {
     const bool strad = a.causal && (min((j + 1) * a.kv_blk, a.N) - 1 >= q_lo);
     const bool forced = j * a.kv_blk < a.forced_prefix_tokens;
     if (strad || forced) lev[j] = 0;
   }
-  __syncthreads();
+  __syncwarp();
   int8_t* mrow = map_ws + (long long)row * a.Nk;
-  for (int j = threadIdx.x; j < a.Nk; j += blockDim.x) {
+  for (int j = lane; j < a.Nk; j += 32) {
     mrow[j] = lev[j];
     if (map_user) map_user[(long long)row * a.Nk + j] = lev[j];
     if (mass_user) mass_user[(long long)row * a.Nk + j] = j < nvis ? expf(z[j] - mx) * inv : 0.f;
   }
-  emit_list(lev, a.Nk, list + (long long)row * a.Nk, counts + row, redi);
+  emit_list_warp(lev, a.Nk, list + (long long)row * a.Nk, counts + row);
 }
 
-__global__ void __launch_bounds__(256) map_to_list_kernel(MaskArgs a,
-                                                          const int8_t* __restrict__ map,
-                                                          int* __restrict__ list,
-                                                          int4* __restrict__ counts) {
+__global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
+                                   const int8_t* __restrict__ map, int* __restrict__ list,
+                                   int4* __restrict__ counts) {
   extern __shared__ __align__(16) unsigned char smem[];
-  int8_t* lev = reinterpret_cast<int8_t*>(smem);
-  __shared__ int redi[33];
-  const int row = blockIdx.x;
-  for (int j = threadIdx.x; j < a.Nk; j += blockDim.x) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * rows_per_cta + warp;
+  if (row >= nrows) return;
+  const int lev_stride = (a.Nk + 15) & ~15;
+  int8_t* lev = reinterpret_cast<int8_t*>(smem) + (size_t)warp * lev_stride;
+  for (int j = lane; j < a.Nk; j += 32) {
     const int8_t v = map[(long long)row * a.Nk + j];
     lev[j] = (v >= 0 && v < kLevels) ? v : (int8_t)-1;
   }
-  __syncthreads();
-  emit_list(lev, a.Nk, list + (long long)row * a.Nk, counts + row, redi);
+  __syncwarp();
+  emit_list_warp(lev, a.Nk, list + (long long)row * a.Nk, counts + row);
 }
 
 int next_pow2(int x) {
@@ -403,25 +369,17 @@ cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, 
 cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, char* ws,
                          cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, scale);
-  const int groups = (L.Nq + 31) / 32;
-  const int base = p.B * p.Hq * groups;
-  int splits = (4 * 148 + base - 1) / base;
-  splits = splits < 1 ? 1 : (splits > L.Nk ? L.Nk : splits);
-  const dim3 grid(base * splits);
+  const int m_tiles = (L.Nq + kSgM - 1) / kSgM;
+  const int n_tiles = (int)((L.rows[3] + kSgN - 1) / kSgN);
+  const long long grid = (long long)p.B * p.Hq * m_tiles * n_tiles;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float* qm = (const float*)(ws + L.qmean);
   const float* k3 = (const float*)(ws + L.k3f);
   float* z = (float*)(ws + L.zlog);
-  const size_t smem = (size_t)2 * kScoreChunk * 8 * p.d * sizeof(float);
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    score_kernel<128><<<grid, 256, smem, st>>>(a, splits, qm, k3, z);
-  } else {
-    e = cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    score_kernel<64><<<grid, 256, smem, st>>>(a, splits, qm, k3, z);
-  }
+  if (p.d == 128)
+    score_kernel<128><<<(unsigned)grid, 256, 0, st>>>(a, m_tiles, n_tiles, qm, k3, z);
+  else
+    score_kernel<64><<<(unsigned)grid, 256, 0, st>>>(a, m_tiles, n_tiles, qm, k3, z);
   return cudaGetLastError();
 }
 
@@ -429,23 +387,32 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
                           int8_t* user_map, float* block_mass, cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, scale);
   const int n2 = next_pow2(L.Nk);
-  const size_t smem = (size_t)n2 * 8 + align256(L.Nk);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  assign_kernel<<<p.B * p.Hq * L.Nq, 256, smem, st>>>(
-      a, n2, (const float*)(ws + L.zlog), (int8_t*)(ws + L.map), user_map, block_mass,
-      (int*)(ws + L.list), (int4*)(ws + L.counts));
+  const size_t per_row = (size_t)n2 * 8 + ((L.Nk + 15) & ~15);
+  int rows_per_cta = (int)((96 * 1024) / per_row);
+  rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 8 ? 8 : rows_per_cta);
+  const size_t smem = per_row * rows_per_cta;
+  cudaError_t e = cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int nrows = p.B * p.Hq * L.Nq;
+  const int grid = (nrows + rows_per_cta - 1) / rows_per_cta;
+  assign_kernel<<<grid, 32 * rows_per_cta, smem, st>>>(
+      a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (int8_t*)(ws + L.map), user_map,
+      block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
   return cudaGetLastError();
 }
 
 cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int8_t* map,
                                char* ws, cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, 0.f);
-  map_to_list_kernel<<<p.B * p.Hq * L.Nq, 256, align256(L.Nk), st>>>(
-      a, map, (int*)(ws + L.list), (int4*)(ws + L.counts));
+  const int rows_per_cta = 8;
+  const size_t smem = (size_t)((L.Nk + 15) & ~15) * rows_per_cta;
+  cudaError_t e = cudaFuncSetAttribute(map_to_list_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int nrows = p.B * p.Hq * L.Nq;
+  map_to_list_kernel<<<(nrows + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, smem, st>>>(
+      a, rows_per_cta, nrows, map, (int*)(ws + L.list), (int4*)(ws + L.counts));
   return cudaGetLastError();
 }
 
