@@ -19,8 +19,9 @@
 //                  level-3 keys, logsumexp over each KV block's keys fused
 //                  into the epilogue.
 //   assign_kernel  one warp per query block: softmax, bitonic sort of packed
-//                  (P, index) keys in shared memory, scan, cut, overrides, and
-//                  the work list (KV block indices grouped by level).
+//                  (P, index) keys (in registers up to 1024 blocks, else in
+//                  shared memory), scan, cut, overrides, and the work list
+//                  (KV block indices grouped by level).
 #include "psa_internal.cuh"
 
 namespace psa {
@@ -242,6 +243,47 @@ __device__ void emit_list_warp(const int8_t* lev, int Nk, int* __restrict__ list
   if (lane == 0) *count_row = make_int4(cnt[0], cnt[1], cnt[2], cnt[3]);
 }
 
+// Bitonic sort of 32*K 64-bit keys held in registers, descending.  Element
+// i = lane*K + r lives in register r of lane `lane`; partners at distance < K
+// are in the same lane, others are exchanged with shuffles.
+template <int K>
+__device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[K]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32 * K; k <<= 1) {
+#pragma unroll
+    for (int sd = k >> 1; sd > 0; sd >>= 1) {
+      if (sd < K) {
+#pragma unroll
+        for (int r = 0; r < K; ++r) {
+          const int rp = r ^ sd;
+          if (rp > r) {
+            const int i = lane * K + r;
+            const bool desc = (i & k) == 0;
+            const unsigned long long a = v[r], b = v[rp];
+            const bool swap = desc ? (a < b) : (a > b);
+            v[r] = swap ? b : a;
+            v[rp] = swap ? a : b;
+          }
+        }
+      } else {
+        const int lx = sd / K;                // partner lane = lane ^ lx
+        const bool upper = (lane & lx) != 0;  // this lane holds the larger index
+#pragma unroll
+        for (int r = 0; r < K; ++r) {
+          const int i = lane * K + r;
+          const bool desc = (i & k) == 0;
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[r], lx);
+          // the lower index keeps the larger key when descending
+          const bool keep_max = desc != upper;
+          v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
+        }
+      }
+    }
+  }
+}
+
+template <int K>
 __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
                               const float* __restrict__ zlog, int8_t* __restrict__ map_ws,
                               int8_t* __restrict__ map_user, float* __restrict__ mass_user,
@@ -269,31 +311,38 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   for (int j = lane; j < nvis; j += 32) part += expf(z[j] - mx);
   const float inv = 1.0f / warp_sum(part);
 
-  for (int i = lane; i < n2; i += 32) {
-    unsigned long long k = 0ull;
-    if (i < nvis) {
-      const float pj = expf(z[i] - mx) * inv;
-      k = ((unsigned long long)__float_as_uint(pj) << 32) | (0xffffffffu - (unsigned)i);
-    }
-    key[i] = k;
-  }
+  auto make_key = [&](int i) -> unsigned long long {
+    if (i >= nvis) return 0ull;
+    const float pj = expf(z[i] - mx) * inv;
+    return ((unsigned long long)__float_as_uint(pj) << 32) | (0xffffffffu - (unsigned)i);
+  };
   for (int j = lane; j < a.Nk; j += 32) lev[j] = -1;
-  __syncwarp();
-
-  // bitonic sort, descending: P high, then lower index first
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int sd = k >> 1; sd > 0; sd >>= 1) {
-      for (int i = lane; i < n2; i += 32) {
-        const int ixj = i ^ sd;
-        if (ixj > i) {
-          const unsigned long long u = key[i], v = key[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (u < v) : (u > v)) { key[i] = v; key[ixj] = u; }
+  if constexpr (K > 0) {
+    unsigned long long v[K];
+#pragma unroll
+    for (int r = 0; r < K; ++r) v[r] = make_key(lane * K + r);
+    warp_bitonic_desc<K>(v);
+#pragma unroll
+    for (int r = 0; r < K; ++r) key[lane * K + r] = v[r];
+  } else {
+    for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
+    __syncwarp();
+    // bitonic sort in shared memory, descending: P high, then lower index first
+    for (int k = 2; k <= n2; k <<= 1) {
+      for (int sd = k >> 1; sd > 0; sd >>= 1) {
+        for (int i = lane; i < n2; i += 32) {
+          const int ixj = i ^ sd;
+          if (ixj > i) {
+            const unsigned long long u = key[i], w = key[ixj];
+            const bool desc = (i & k) == 0;
+            if (desc ? (u < w) : (u > w)) { key[i] = w; key[ixj] = u; }
+          }
         }
+        __syncwarp();
       }
-      __syncwarp();
     }
   }
+  __syncwarp();
 
   // exclusive running mass in rank order (lanes take contiguous rank ranges)
   const int per = (nvis + 31) / 32;
@@ -386,20 +435,30 @@ cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, ch
 cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, char* ws,
                           int8_t* user_map, float* block_mass, cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, scale);
-  const int n2 = next_pow2(L.Nk);
+  const int n2 = next_pow2(L.Nk < 32 ? 32 : L.Nk);
   const size_t per_row = (size_t)n2 * 8 + ((L.Nk + 15) & ~15);
   int rows_per_cta = (int)((96 * 1024) / per_row);
   rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 8 ? 8 : rows_per_cta);
   const size_t smem = per_row * rows_per_cta;
-  cudaError_t e = cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
   const int nrows = p.B * p.Hq * L.Nq;
   const int grid = (nrows + rows_per_cta - 1) / rows_per_cta;
-  assign_kernel<<<grid, 32 * rows_per_cta, smem, st>>>(
-      a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (int8_t*)(ws + L.map), user_map,
-      block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
-  return cudaGetLastError();
+  auto go = [&](auto kern) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 32 * rows_per_cta, smem, st>>>(
+        a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (int8_t*)(ws + L.map), user_map,
+        block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
+    return cudaGetLastError();
+  };
+  switch (n2) {   // keys per lane for the register sort; larger rows sort in shared memory
+    case 32: return go(assign_kernel<1>);
+    case 64: return go(assign_kernel<2>);
+    case 128: return go(assign_kernel<4>);
+    case 256: return go(assign_kernel<8>);
+    case 512: return go(assign_kernel<16>);
+    case 1024: return go(assign_kernel<32>);
+    default: return go(assign_kernel<0>);
+  }
 }
 
 cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int8_t* map,
