@@ -92,7 +92,7 @@ constexpr int kSgPad = 4;      // row padding of the transposed shared tiles
 // double-buffered through registers: per k-step a thread reads 3 x 16 bytes
 // and issues 32 FMA.
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int m_tiles, int n_tiles,
+__global__ void __launch_bounds__(256, 3) score_kernel(MaskArgs a, int m_tiles, int n_tiles,
                                                     const float* __restrict__ qmean,
                                                     const float* __restrict__ k3f,
                                                     float* __restrict__ zlog) {
@@ -110,25 +110,30 @@ __global__ void __launch_bounds__(256) score_kernel(MaskArgs a, int m_tiles, int
   const float* Ag = qmean + (long long)bhq * a.Nq * D;
   const float* Bg = k3f + (long long)bhk * rows3 * D;
   const int tid = threadIdx.x;
-  const int tm = tid >> 4, tn = tid & 15;
+  // a warp covers 8 query-block groups x 4 KV blocks, so each k-step reads
+  // 128 + 128 bytes of shared memory per warp for its 32 FMA per thread
+  const int lane = tid & 31, wid = tid >> 5;
+  const int tm = (wid >> 2) * 8 + (lane >> 2), tn = (wid & 3) * 4 + (lane & 3);
 
-  // global -> register staging: A 64x16 (one float4 per thread), B 128x16 (two)
-  const int ar = tid >> 2, ak = (tid & 3) * 4;
-  const int br0 = tid >> 2, br1 = br0 + 64, bk = (tid & 3) * 4;
+  // global -> register staging: A 64x16 (one float4 per thread), B 128x16
+  // (two).  Consecutive threads take consecutive rows, so the transposed
+  // shared-memory stores of a warp hit 32 different banks.
+  const int ar = tid & 63, ak = (tid >> 6) * 4;
+  const int br0 = tid & 127, br1 = br0, bk = (tid >> 7) * 4;
   float4 ra, rb0, rb1;
   auto load = [&](int k0) {
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     ra = (m0 + ar < a.Nq) ? *reinterpret_cast<const float4*>(Ag + (long long)(m0 + ar) * D + k0 + ak) : zero;
     rb0 = (n0 + br0 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br0) * D + k0 + bk)) : zero;
-    rb1 = (n0 + br1 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br1) * D + k0 + bk)) : zero;
+    rb1 = (n0 + br1 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br1) * D + k0 + bk + 8)) : zero;
   };
   auto store = [&](int buf) {
     As[buf][ak + 0][ar] = ra.x; As[buf][ak + 1][ar] = ra.y;
     As[buf][ak + 2][ar] = ra.z; As[buf][ak + 3][ar] = ra.w;
     Bs[buf][bk + 0][br0] = rb0.x; Bs[buf][bk + 1][br0] = rb0.y;
     Bs[buf][bk + 2][br0] = rb0.z; Bs[buf][bk + 3][br0] = rb0.w;
-    Bs[buf][bk + 0][br1] = rb1.x; Bs[buf][bk + 1][br1] = rb1.y;
-    Bs[buf][bk + 2][br1] = rb1.z; Bs[buf][bk + 3][br1] = rb1.w;
+    Bs[buf][bk + 8][br1] = rb1.x; Bs[buf][bk + 9][br1] = rb1.y;
+    Bs[buf][bk + 10][br1] = rb1.z; Bs[buf][bk + 11][br1] = rb1.w;
   };
 
   float acc[4][8];
@@ -249,34 +254,35 @@ __device__ void emit_list_warp(const int8_t* lev, int Nk, int* __restrict__ list
 template <int K>
 __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[K]) {
   const int lane = threadIdx.x & 31;
-#pragma unroll
+#pragma unroll 1
   for (int k = 2; k <= 32 * K; k <<= 1) {
+    // stages whose partner is in another lane (distance >= K)
+#pragma unroll 1
+    for (int sd = k >> 1; sd >= K; sd >>= 1) {
+      const int lx = sd / K;                // partner lane = lane ^ lx
+      const bool upper = (lane & lx) != 0;  // this lane holds the larger index
 #pragma unroll
-    for (int sd = k >> 1; sd > 0; sd >>= 1) {
-      if (sd < K) {
+      for (int r = 0; r < K; ++r) {
+        const bool desc = ((lane * K + r) & k) == 0;
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[r], lx);
+        const bool keep_max = desc != upper;  // descending pairs keep the max at the lower index
+        v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
+      }
+    }
+    // stages inside a lane (distance < K), unrolled so registers stay static
+#pragma unroll
+    for (int sd = K / 2; sd > 0; sd >>= 1) {
+      if (sd < k) {
 #pragma unroll
         for (int r = 0; r < K; ++r) {
           const int rp = r ^ sd;
           if (rp > r) {
-            const int i = lane * K + r;
-            const bool desc = (i & k) == 0;
-            const unsigned long long a = v[r], b = v[rp];
-            const bool swap = desc ? (a < b) : (a > b);
-            v[r] = swap ? b : a;
-            v[rp] = swap ? a : b;
+            const bool desc = ((lane * K + r) & k) == 0;
+            const unsigned long long x = v[r], y = v[rp];
+            const bool swap = desc ? (x < y) : (x > y);
+            v[r] = swap ? y : x;
+            v[rp] = swap ? x : y;
           }
-        }
-      } else {
-        const int lx = sd / K;                // partner lane = lane ^ lx
-        const bool upper = (lane & lx) != 0;  // this lane holds the larger index
-#pragma unroll
-        for (int r = 0; r < K; ++r) {
-          const int i = lane * K + r;
-          const bool desc = (i & k) == 0;
-          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[r], lx);
-          // the lower index keeps the larger key when descending
-          const bool keep_max = desc != upper;
-          v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
         }
       }
     }
@@ -293,8 +299,9 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   const int row = blockIdx.x * rows_per_cta + warp;
   if (row >= nrows) return;                 // whole warp; no block barriers below
   const int lev_stride = (a.Nk + 15) & ~15;
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem) + (size_t)warp * n2;
-  int8_t* lev = reinterpret_cast<int8_t*>(smem + (size_t)rows_per_cta * n2 * 8) +
+  const size_t key_bytes = K > 0 ? 0 : (size_t)n2 * 8;       // keys in registers when K > 0
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem) + (size_t)warp * (key_bytes / 8);
+  int8_t* lev = reinterpret_cast<int8_t*>(smem + (size_t)rows_per_cta * key_bytes) +
                 (size_t)warp * lev_stride;
 
   const int qa = row % a.Nq;
@@ -310,20 +317,40 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   float part = 0.f;
   for (int j = lane; j < nvis; j += 32) part += expf(z[j] - mx);
   const float inv = 1.0f / warp_sum(part);
-
   auto make_key = [&](int i) -> unsigned long long {
     if (i >= nvis) return 0ull;
     const float pj = expf(z[i] - mx) * inv;
     return ((unsigned long long)__float_as_uint(pj) << 32) | (0xffffffffu - (unsigned)i);
   };
   for (int j = lane; j < a.Nk; j += 32) lev[j] = -1;
+
+  // rank by P descending (ties to the lower index), exclusive running mass,
+  // level = first tau the running mass is below
   if constexpr (K > 0) {
-    unsigned long long v[K];
+    // sorted keys stay in registers: lane L holds ranks L*K .. L*K + K - 1
+    unsigned long long v[K > 0 ? K : 1];
 #pragma unroll
     for (int r = 0; r < K; ++r) v[r] = make_key(lane * K + r);
     warp_bitonic_desc<K>(v);
+    __syncwarp();                          // lev[] initialised by all lanes
+    float mine = 0.f;
 #pragma unroll
-    for (int r = 0; r < K; ++r) key[lane * K + r] = v[r];
+    for (int r = 0; r < K; ++r)
+      if (lane * K + r < nvis) mine += __uint_as_float((unsigned)(v[r] >> 32));
+    float total;
+    float c = warp_excl_scan(mine, &total);
+#pragma unroll
+    for (int r = 0; r < K; ++r) {
+      if (lane * K + r < nvis) {
+        const int j = (int)(0xffffffffu - (unsigned)(v[r] & 0xffffffffu));
+        int l = -1;
+#pragma unroll
+        for (int t = kLevels - 1; t >= 0; --t)
+          if (c < a.tau[t]) l = t;
+        lev[j] = (int8_t)l;
+        c += __uint_as_float((unsigned)(v[r] >> 32));
+      }
+    }
   } else {
     for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
     __syncwarp();
@@ -341,25 +368,22 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
         __syncwarp();
       }
     }
-  }
-  __syncwarp();
-
-  // exclusive running mass in rank order (lanes take contiguous rank ranges)
-  const int per = (nvis + 31) / 32;
-  const int r0 = lane * per, r1 = min(nvis, r0 + per);
-  float mine = 0.f;
-  for (int r = r0; r < r1; ++r) mine += __uint_as_float((unsigned)(key[r] >> 32));
-  float total;
-  float c = warp_excl_scan(mine, &total);
-  for (int r = r0; r < r1; ++r) {
-    const float pr = __uint_as_float((unsigned)(key[r] >> 32));
-    const int j = (int)(0xffffffffu - (unsigned)(key[r] & 0xffffffffu));
-    int l = -1;
+    const int per = (nvis + 31) / 32;       // lanes take contiguous rank ranges
+    const int r0 = lane * per, r1 = min(nvis, r0 + per);
+    float mine = 0.f;
+    for (int r = r0; r < r1; ++r) mine += __uint_as_float((unsigned)(key[r] >> 32));
+    float total;
+    float c = warp_excl_scan(mine, &total);
+    for (int r = r0; r < r1; ++r) {
+      const float pr = __uint_as_float((unsigned)(key[r] >> 32));
+      const int j = (int)(0xffffffffu - (unsigned)(key[r] & 0xffffffffu));
+      int l = -1;
 #pragma unroll
-    for (int t = kLevels - 1; t >= 0; --t)
-      if (c < a.tau[t]) l = t;
-    lev[j] = (int8_t)l;
-    c += pr;
+      for (int t = kLevels - 1; t >= 0; --t)
+        if (c < a.tau[t]) l = t;
+      lev[j] = (int8_t)l;
+      c += pr;
+    }
   }
   __syncwarp();
   // overrides: causal diagonal -> 0, forced prefix -> 0 (visible blocks only)
@@ -436,9 +460,10 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
                           int8_t* user_map, float* block_mass, cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, scale);
   const int n2 = next_pow2(L.Nk < 32 ? 32 : L.Nk);
-  const size_t per_row = (size_t)n2 * 8 + ((L.Nk + 15) & ~15);
+  const bool in_regs = n2 <= 1024;          // register sort; larger rows sort in shared memory
+  const size_t per_row = (in_regs ? 0 : (size_t)n2 * 8) + ((L.Nk + 15) & ~15);
   int rows_per_cta = (int)((96 * 1024) / per_row);
-  rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 8 ? 8 : rows_per_cta);
+  rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 2 ? 2 : rows_per_cta);
   const size_t smem = per_row * rows_per_cta;
   const int nrows = p.B * p.Hq * L.Nq;
   const int grid = (nrows + rows_per_cta - 1) / rows_per_cta;
