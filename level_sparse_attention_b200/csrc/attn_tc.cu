@@ -13,9 +13,10 @@
 // carries their softmax mass.
 //
 // Persistent CTAs (one per SM) walk the query blocks; per query block, 10 warps:
-//   warp 0     TMA producer: Q once; per tile, one 2-D box per sub-block and
-//              64-column half for K and for V (the box height is the level's
-//              sub-block height), plus a per-key bias / position table.
+//   warp 0     TMA producer for Q and K: Q once per query block; per tile, one
+//              2-D box per sub-block and 64-column half (the box height is the
+//              level's sub-block height), plus the tile's key bias table.
+//   warp 10    TMA producer for V, the same boxes into the V ring.
 //   warp 1     TMEM allocator and single-thread tcgen05.mma issuer:
 //              S[t%2] = Q K_t^T (SS form), then O += P_t V_t with P read from
 //              TMEM (TS form); commits signal the softmax and free stages.
@@ -38,7 +39,9 @@ namespace {
 
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per packed tile
-constexpr int kThreads = 320;     // producer, MMA, 2 softmax warpgroups
+constexpr int kSoftGroups = 2;    // softmax warpgroups sharing each tile (64 keys each)
+constexpr int kVWarp = 2 + 4 * kSoftGroups;        // the V producer, after the softmax warps
+constexpr int kThreads = 96 + 128 * kSoftGroups;   // K producer, MMA, softmax, V producer
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -60,9 +63,9 @@ struct Cfg {
   static constexpr int OFF_META = OFF_V + VSTAGES * KV_BYTES;   // per table: bias[128], kpos[128]
   static constexpr int META_BYTES = 128 + 1024;                // chunk biases, flag, per-key tables
   static constexpr int OFF_BAR = OFF_META + MSTAGES * META_BYTES;
-  static constexpr int OFF_XCH = OFF_BAR + 512;                 // softmax pair exchange [2][2][128]
-  static constexpr int OFF_LIST = OFF_XCH + 2048;               // the query block's work list
-  static constexpr int SMEM = OFF_LIST + kListCache * 4 + 1024; // + slack for 1024 alignment
+  static constexpr int OFF_XCH = OFF_BAR + 512;                 // softmax exchange [2][groups][128]
+  static constexpr int OFF_LIST = OFF_XCH + 2 * kSoftGroups * 512;   // the query block's work list
+  static constexpr int SMEM = OFF_LIST + 2 * kListCache * 4 + 1024;   // two list copies + slack
 };
 
 struct __align__(64) TcParams {
@@ -270,6 +273,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       PSA_W8(0), PSA_W8(8), PSA_W8(16), PSA_W8(24)
       : "memory");
 }
+#define PSA_R4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
+#define PSA_W4(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3])
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : PSA_R4(0), PSA_R4(4), PSA_R4(8), PSA_R4(12)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      PSA_W4(0), PSA_W4(4), PSA_W4(8), PSA_W4(12)
+      : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 64) {
+    tmem_ld32(taddr, r);
+    tmem_ld32(taddr + 32, r + 32);
+  } else if constexpr (N == 32) {
+    tmem_ld32(taddr, r);
+  } else {
+    tmem_ld16(taddr, r);
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 32) tmem_st32(taddr, r); else tmem_st16(taddr, r);
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -370,10 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     mbar_init(bar(B_QEMPTY), 1);
     for (int s = 0; s < KS; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
-    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 8); }
+    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 4 * kSoftGroups); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PFULL + i), 256);
+      mbar_init(bar(B_PFULL + i), 128 * kSoftGroups);
       mbar_init(bar(B_ODONE + i), 1);
     }
     mbar_init(bar(B_FINAL), 1);
@@ -402,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t T_S = tmem, T_P = tmem + 256, T_O = tmem + 384;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int gk = 0, gv = 0, iq = 0;
+    // ---------------------------------------------------- K / Q producer
+    int gk = 0, iq = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
       const RowWork w = row_work(p.counts[item]);
@@ -418,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       __syncwarp();
       for (int i = lane; i < n_ent; i += 32) lcache[i] = __ldg(lrow + i);
       __syncwarp();
-      TileEntry cur = tile_entry(w, lrow, lcache, 0, lane), prev = cur;
+      TileEntry cur = tile_entry(w, lrow, lcache, 0, lane);
       if (iq > 0 && !warp_wait(bar(B_QEMPTY), (iq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
       if (lane == 0) {
         mbar_expect_tx(bar(B_QFULL), C::Q_BYTES);
@@ -427,21 +461,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                       qa * kBM, bhq);
       }
       ++iq;
-      for (int t = 0; t <= T; ++t) {
+      for (int t = 0; t < T; ++t) {
         // the next tile's list entries are loaded before this tile's waits
         const TileEntry nxt = t + 1 < T ? tile_entry(w, lrow, lcache, t + 1, lane) : cur;
-        if (t < T) {
+        {
           // K of tile t, and its per-key bias / position table
           const int s = gk % KS, ms = gk % MS;
           if (gk >= KS && !warp_wait(bar(B_KEMPTY + s), ((gk / KS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
           if (gk >= MS && !warp_wait(bar(B_MEMPTY + ms), ((gk / MS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
           const int n_in = __popc(__ballot_sync(0xffffffffu, cur.in_tile));
-          int bytes = cur.in_tile ? cur.R * D * 2 : 0;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+          // every entry fills exactly its R rows, so the tile carries
+          // min(128, keys - 128 t) keys
+          const int bytes = min(kBN, w.b4 - t * kBN) * D * 2;
           // Per-key bias table of this tile.  Usually every key of an 8-key
           // chunk has bias = its level (log2 of the pool factor), so 16 chunk
-          // values describe the tile.  Tiles holding the ragged last KV block
+          // values describe the tile, read off the level boundaries of the
+          // packed key sequence.  Tiles holding the ragged last KV block
           // (partial groups, rows past the end) or, causally, a block that
           // straddles the diagonal (token positions) get a full per-key table.
           unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
@@ -453,19 +488,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                (p.causal && cur.l == 0 &&
                                 (cur.j + 1) * 64 - 1 >= qa * kBM));
           const bool slow = __any_sync(0xffffffffu, special);
-          const int col = slow ? 4 * lane : 8 * (lane & 15);
-          int owner = 0;
-          for (int i = 1; i < n_in; ++i)
-            if (__shfl_sync(0xffffffffu, cur.r0, i) <= col) owner = i;
-          const int oj = __shfl_sync(0xffffffffu, cur.j, owner);
-          const int ol = __shfl_sync(0xffffffffu, cur.l, owner);
-          const int oR = __shfl_sync(0xffffffffu, cur.R, owner);
-          const int or0 = __shfl_sync(0xffffffffu, cur.r0, owner);
-          const bool live = n_in > 0 && col < or0 + oR;   // false past the last entry
           if (!slow) {
-            if (lane < 16) cbias[lane] = live ? (float)ol : -INFINITY;
+            if (lane < 16) {
+              const int off = t * kBN + 8 * lane;
+              const int lvl = (off >= w.b1) + (off >= w.b2) + (off >= w.b3);
+              cbias[lane] = off < w.b4 ? (float)lvl : -INFINITY;
+            }
             if (lane == 16) *mflag = 0;
           } else {
+            const int col = 4 * lane;
+            int owner = 0;
+            for (int i = 1; i < n_in; ++i)
+              if (__shfl_sync(0xffffffffu, cur.r0, i) <= col) owner = i;
+            const int oj = __shfl_sync(0xffffffffu, cur.j, owner);
+            const int ol = __shfl_sync(0xffffffffu, cur.l, owner);
+            const int oR = __shfl_sync(0xffffffffu, cur.R, owner);
+            const int or0 = __shfl_sync(0xffffffffu, cur.r0, owner);
+            const bool live = n_in > 0 && col < or0 + oR;   // false past the last entry
             float bias[4];
             int kpos[4];
 #pragma unroll
@@ -491,24 +530,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
           ++gk;
         }
-        if (t >= 1) {
-          // V of tile t - 1 (same entries as its K)
-          const int s = gv % VS;
-          if (gv >= VS && !warp_wait(bar(B_VEMPTY + s), ((gv / VS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          int bytes = prev.in_tile ? prev.R * D * 2 : 0;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-          if (lane == 0) mbar_expect_tx(bar(B_VFULL + s), bytes);
-          __syncwarp();
-          if (prev.in_tile) {
-            const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + prev.r0 * 128;
-            for (int h = 0; h < C::HALVES; ++h)
-              tma_load_3d(vdst + h * C::HALF, &p.tv[prev.l], bar(B_VFULL + s), h * 64,
-                          prev.j * prev.R, bhk);
-          }
-          ++gv;
+        cur = nxt;
+      }
+    }
+  } else if (warp == kVWarp) {
+    // ------------------------------------------------------------ V producer
+    int gv = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+      const RowWork w = row_work(p.counts[item]);
+      const int T = w.tiles;
+      if (T == 0) continue;
+      const int bhq = item / p.Nq;
+      const int bhk = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / (p.Hq / p.Hkv);
+      const int* lrow = p.list + (long long)item * p.Nk;
+      int* lcache = reinterpret_cast<int*>(smem + C::OFF_LIST + kListCache * 4);
+      const int n_ent = min(w.f4, kListCache);
+      __syncwarp();
+      for (int i = lane; i < n_ent; i += 32) lcache[i] = __ldg(lrow + i);
+      __syncwarp();
+      TileEntry cur = tile_entry(w, lrow, lcache, 0, lane);
+      for (int t = 0; t < T; ++t) {
+        const TileEntry nxt = t + 1 < T ? tile_entry(w, lrow, lcache, t + 1, lane) : cur;
+        const int s = gv % VS;
+        if (gv >= VS && !warp_wait(bar(B_VEMPTY + s), ((gv / VS) + 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        const int bytes = min(kBN, w.b4 - t * kBN) * D * 2;
+        if (lane == 0) mbar_expect_tx(bar(B_VFULL + s), bytes);
+        __syncwarp();
+        if (cur.in_tile) {
+          const uint32_t vdst = sbase + C::OFF_V + s * C::KV_BYTES + cur.r0 * 128;
+          for (int h = 0; h < C::HALVES; ++h)
+            tma_load_3d(vdst + h * C::HALF, &p.tv[cur.l], bar(B_VFULL + s), h * 64,
+                        cur.j * cur.R, bhk);
         }
-        prev = cur;
+        ++gv;
         cur = nxt;
       }
     }
@@ -567,27 +622,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else {
     // --------------------------------------------------------------- softmax
-    // Two warpgroups share every row: group hg takes keys [64*hg, 64*hg + 64)
-    // of each tile and O columns [hg*D/2, (hg+1)*D/2).  The pair of warps that
-    // own the same 32 rows (same TMEM lane quadrant) exchange their partial
-    // row maxima every tile through shared memory and a 64-thread named
-    // barrier, so both keep the same running max; the partial row sums are
-    // added at the end.  Both warps of a pair always take the same number of
-    // barriers, also when a wait has timed out, so the barrier cannot hang.
-    constexpr int HD = D / 2;
-    constexpr int NPOLY = 24;      // columns of each 64 whose 2^x runs on the FMA pipes
+    // kSoftGroups warpgroups share every row: group hg takes keys
+    // [KW*hg, KW*hg + KW) of each tile and O columns [hg*HD, (hg+1)*HD).  The
+    // warps that own the same 32 rows (same TMEM lane quadrant) exchange
+    // their partial row maxima every tile through shared memory and a named
+    // barrier, so all keep the same running max; partial row sums are added
+    // at the end.  Every warp takes the same number of barriers on every path
+    // (also after a timed-out wait), so the barrier cannot hang.
+    constexpr int NG = kSoftGroups;
+    constexpr int KW = kBN / NG;        // keys per group and tile
+    constexpr int HD = D / NG;          // O columns per group
+    constexpr int OC = HD < 32 ? HD : 32;
+    constexpr int NPOLY = (KW * 3) / 8; // keys per group whose 2^x runs on the FMA pipes
     const int hg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][2][128]
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][NG][128]
     int nx = 0;                                                 // exchanges so far
-    auto exchange = [&](float v) -> float {   // returns the partner's value
-      float* buf = xch + (nx & 1) * 256;
+    // writes v, returns the NG values of this row (group order)
+    auto exchange = [&](float v, float (&all)[NG]) {
+      float* buf = xch + (nx & 1) * (NG * 128);
       buf[hg * 128 + r] = v;
-      asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "r"(32 * NG) : "memory");
       ++nx;
-      return buf[(1 - hg) * 128 + r];
+#pragma unroll
+      for (int i = 0; i < NG; ++i) all[i] = buf[i * 128 + r];
     };
     const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
     int g = 0;
@@ -601,68 +661,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int gt = g + t, bb = gt & 1, ms = gt % MS;
         ok = ok && warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) &&
              warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err);
-        float x[64];
+        float x[KW];
         float mt = -INFINITY;
         if (ok) {
           tc_fence_after();
           const unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
           const bool slow = *reinterpret_cast<const int*>(mt_base + 64) != 0;
-          const float* cb = reinterpret_cast<const float*>(mt_base) + 8 * hg;
-          const float* mbias = reinterpret_cast<const float*>(mt_base + 128) + 64 * hg;
-          const int* mpos = reinterpret_cast<const int*>(mt_base + 128 + 512) + 64 * hg;
-          const float4 cb0 = *reinterpret_cast<const float4*>(cb);
-          const float4 cb1 = *reinterpret_cast<const float4*>(cb + 4);
-          const float cbv[8] = {cb0.x, cb0.y, cb0.z, cb0.w, cb1.x, cb1.y, cb1.z, cb1.w};
-          const uint32_t sa = T_S + bb * 128 + lane_off + 64 * hg;
-          tmem_ld32(sa, reinterpret_cast<uint32_t*>(x));
+          const float* cb = reinterpret_cast<const float*>(mt_base) + (KW / 8) * hg;
+          const float* mbias = reinterpret_cast<const float*>(mt_base + 128) + KW * hg;
+          const int* mpos = reinterpret_cast<const int*>(mt_base + 128 + 512) + KW * hg;
+          tmem_ldn<KW>(T_S + bb * 128 + lane_off + KW * hg, reinterpret_cast<uint32_t*>(x));
+          float cbv[KW / 8];
+#pragma unroll
+          for (int i = 0; i < KW / 8; ++i) cbv[i] = cb[i];
           tmem_ld_wait();
-          reg_fence<32>(reinterpret_cast<uint32_t*>(x));
-          tmem_ld32(sa + 32, reinterpret_cast<uint32_t*>(x + 32));   // in flight during the first half
+          reg_fence<KW>(reinterpret_cast<uint32_t*>(x));
           float mx0 = -INFINITY, mx1 = -INFINITY;
+          if (!slow) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            if (half == 1) {
-              tmem_ld_wait();
-              reg_fence<32>(reinterpret_cast<uint32_t*>(x + 32));
+            for (int c = 0; c < KW; c += 4) {
+              const float b = cbv[c >> 3];
+              const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b, b));
+              const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b, b));
+              f2unpack(v01, x[c], x[c + 1]);
+              f2unpack(v23, x[c + 2], x[c + 3]);
+              mx0 = fmax3(mx0, x[c], x[c + 1]);
+              mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
             }
-            if (!slow) {
+          } else {
 #pragma unroll
-              for (int c = half * 32; c < half * 32 + 32; c += 4) {
-                const float b = cbv[c >> 3];
-                const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b, b));
-                const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b, b));
-                f2unpack(v01, x[c], x[c + 1]);
-                f2unpack(v23, x[c + 2], x[c + 3]);
-                mx0 = fmax3(mx0, x[c], x[c + 1]);
-                mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+            for (int c = 0; c < KW; c += 4) {
+              const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
+              const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b4.x, b4.y));
+              const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b4.z, b4.w));
+              f2unpack(v01, x[c], x[c + 1]);
+              f2unpack(v23, x[c + 2], x[c + 3]);
+              if (p.causal) {
+                const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
+                if (qpos < k4.x) x[c] = -INFINITY;
+                if (qpos < k4.y) x[c + 1] = -INFINITY;
+                if (qpos < k4.z) x[c + 2] = -INFINITY;
+                if (qpos < k4.w) x[c + 3] = -INFINITY;
               }
-            } else {
-#pragma unroll
-              for (int c = half * 32; c < half * 32 + 32; c += 4) {
-                const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
-                const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b4.x, b4.y));
-                const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b4.z, b4.w));
-                f2unpack(v01, x[c], x[c + 1]);
-                f2unpack(v23, x[c + 2], x[c + 3]);
-                if (p.causal) {
-                  const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
-                  if (qpos < k4.x) x[c] = -INFINITY;
-                  if (qpos < k4.y) x[c + 1] = -INFINITY;
-                  if (qpos < k4.z) x[c + 2] = -INFINITY;
-                  if (qpos < k4.w) x[c + 3] = -INFINITY;
-                }
-                mx0 = fmax3(mx0, x[c], x[c + 1]);
-                mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
-              }
+              mx0 = fmax3(mx0, x[c], x[c + 1]);
+              mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
             }
           }
           mt = fmaxf(mx0, mx1);
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
         }
-        const float other = exchange(mt);
+        float parts[NG];
+        exchange(mt, parts);
         if (!ok) continue;
-        mt = hg == 0 ? fmaxf(mt, other) : fmaxf(other, mt);
+        mt = parts[0];
+#pragma unroll
+        for (int i = 1; i < NG; ++i) mt = fmaxf(mt, parts[i]);
         const float m_new = fmaxf(m, mt);
         const bool need = m_new > m + kRescaleLog2;     // false while both are -inf
         if (__any_sync(0xffffffffu, need)) {
@@ -673,14 +727,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (ok) {
               tc_fence_after();
 #pragma unroll
-              for (int c0 = 0; c0 < HD; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(T_O + lane_off + hg * HD + c0, o);
+              for (int c0 = 0; c0 < HD; c0 += OC) {
+                uint32_t o[OC];
+                tmem_ldn<OC>(T_O + lane_off + hg * HD + c0, o);
                 tmem_ld_wait();
-                reg_fence<32>(o);
+                reg_fence<OC>(o);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                tmem_st32(T_O + lane_off + hg * HD + c0, o);
+                for (int i = 0; i < OC; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+                tmem_stn<OC>(T_O + lane_off + hg * HD + c0, o);
               }
             }
           }
@@ -691,13 +745,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float m_base = m == -INFINITY ? 0.f : m;
         const uint64_t nm2 = f2pack(-m_base, -m_base);
         uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
-        uint32_t pk[32];
+        uint32_t pk[KW / 2];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
+        for (int c = 0; c < KW; c += 2) {
           float p0, p1;
-          const uint64_t d = fadd2(f2pack(x[c], x[c + 1]), nm2);
+          const uint64_t dd = fadd2(f2pack(x[c], x[c + 1]), nm2);
           float d0, d1;
-          f2unpack(d, d0, d1);
+          f2unpack(dd, d0, d1);
           if (c < NPOLY) {
             exp2_poly2(d0, d1, p0, p1);
           } else {
@@ -709,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
           pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
         }
-        tmem_st32(T_P + bb * 64 + lane_off + 32 * hg, pk);
+        tmem_stn<KW / 2>(T_P + bb * 64 + lane_off + (KW / 2) * hg, pk);
         float a0, a1, a2, a3;
         f2unpack(acc0, a0, a1);
         f2unpack(acc1, a2, a3);
@@ -719,8 +773,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mbar_arrive(bar(B_PFULL + bb));
       }
       // epilogue of this query block: full row sum, then this group's O columns
-      const float other = exchange(lsum);
-      const float ltot = hg == 0 ? lsum + other : other + lsum;
+      float parts[NG];
+      exchange(lsum, parts);
+      float ltot = parts[0];
+#pragma unroll
+      for (int i = 1; i < NG; ++i) ltot += parts[i];
       const bool row_ok = qpos < p.N;
       const bool keys = m > -INFINITY;                  // the row kept at least one key
       const float inv = keys ? 1.f / ltot : 0.f;
@@ -730,27 +787,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                     abort_flag, p.err);
       if (have_o) tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t o[32];
+      for (int c0 = 0; c0 < HD; c0 += OC) {
+        uint32_t o[OC];
         if (have_o) {
-          tmem_ld32(T_O + lane_off + hg * HD + c0, o);
+          tmem_ldn<OC>(T_O + lane_off + hg * HD + c0, o);
           tmem_ld_wait();
-          reg_fence<32>(o);
+          reg_fence<OC>(o);
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int i = 0; i < OC; ++i) o[i] = 0u;
         }
         if (row_ok) {
-          uint32_t pk[16];
+          uint32_t pk[OC / 2];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < OC / 2; ++i) {
             __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
                                                       __uint_as_float(o[2 * i + 1]) * inv);
             pk[i] = *reinterpret_cast<uint32_t*>(&hh);
           }
           uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+          for (int i = 0; i < OC / 8; ++i)
             d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
