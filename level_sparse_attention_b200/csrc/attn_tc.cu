@@ -572,46 +572,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_bf16(kBM, kBN, false);
       constexpr uint32_t ID_PV = idesc_bf16(kBM, D, true);
+      static_assert(kBM * 128 == C::HALF, "Q and K tiles share one half-tile layout");
+      const uint64_t qdesc0 = sdesc(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t kdesc0 = sdesc(sbase + C::OFF_K, 16, 1024);
+      const uint64_t vdesc0 = sdesc(sbase + C::OFF_V, C::HALF, 1024);
       bool ok = true;
       auto issue_pv = [&](int u, bool first) -> bool {
         const int s = u % VS, bb = u & 1;
         if (!wait_bar(bar(B_PFULL + bb), (u >> 1) & 1, abort_flag, p.err)) return false;
         if (!wait_bar(bar(B_VFULL + s), (u / VS) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
-        const uint32_t vb = sbase + C::OFF_V + s * C::KV_BYTES;
+        const uint64_t vd = vdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
+        const uint32_t dP = T_P + bb * 64;
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k)
-          mma_ts(T_O, T_P + bb * 64 + k * 8, sdesc(vb + k * 2048, C::HALF, 1024), ID_PV,
+          mma_ts(T_O, dP + k * 8, vd + (uint64_t)(k * (2048 >> 4)), ID_PV,
                  (first && k == 0) ? 0u : 1u);
         mma_commit(bar(B_ODONE + bb));
         mma_commit(bar(B_VEMPTY + s));
         return true;
       };
+      // QK^T of tile u into S[u % 2].  That buffer was last read by the
+      // softmax of tile u - 2, which finished before P(u - 2) was ready, and
+      // PV(u - 2) (issued before this call) waited for P(u - 2).
+      auto issue_qk = [&](int u) -> bool {
+        const int s = u % KS, bb = u & 1;
+        if (!wait_bar(bar(B_KFULL + s), (u / KS) & 1, abort_flag, p.err)) return false;
+        tc_fence_after();
+        // descriptors advance by adding the byte offset / 16 to the start-address field
+        const uint64_t kd = kdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
+        const uint32_t dS = T_S + bb * 128;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          constexpr uint32_t kHalfStep = C::HALF >> 4;   // same layout for Q and K halves
+          const uint64_t off = (uint64_t)((k >> 2) * kHalfStep + (k & 3) * 2);
+          mma_ss(dS, qdesc0 + off, kd + off, ID_QK, k > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(B_SFULL + bb));
+        mma_commit(bar(B_KEMPTY + s));
+        return true;
+      };
+      // Order per query block: QK(0), then for each tile t >= 1: QK(t), PV(t - 1);
+      // finally PV(T - 1).  QK^T of the next tile runs while the softmax of the
+      // current one works.
       int g = 0, iq = 0;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
         if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
         ++iq;
-        for (int t = 0; t < T; ++t) {
-          const int gk = g + t, s = gk % KS, bb = gk & 1;
-          if (!wait_bar(bar(B_KFULL + s), (gk / KS) & 1, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = sbase + C::OFF_K + s * C::KV_BYTES;
-          const uint32_t qb = sbase + C::OFF_Q;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t koff = (k >> 2) * C::HALF + (k & 3) * 32;
-            const uint32_t qoff = (k >> 2) * (kBM * 128) + (k & 3) * 32;
-            mma_ss(T_S + bb * 128, sdesc(qb + qoff, 16, 1024), sdesc(kb + koff, 16, 1024), ID_QK,
-                   k > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(B_SFULL + bb));
-          mma_commit(bar(B_KEMPTY + s));
-          if (t == T - 1) mma_commit(bar(B_QEMPTY));
-          if (t >= 1 && !issue_pv(gk - 1, t == 1)) { ok = false; break; }
+        for (int t = 0; ok && t < T; ++t) {
+          ok = issue_qk(g + t);
+          if (ok && t == T - 1) mma_commit(bar(B_QEMPTY));
+          if (ok && t >= 1) ok = issue_pv(g + t - 1, t == 1);
         }
-        if (!ok || !issue_pv(g + T - 1, T == 1)) { ok = false; break; }
+        if (ok) ok = issue_pv(g + T - 1, T == 1);
+        if (!ok) break;
         g += T;
       }
       // drain: every MMA issued so far completes before TMEM is released
@@ -763,6 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
           pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
         }
+        // P(gt - 2) in this buffer has been consumed: S(gt) was committed after
+        // PV(gt - 2) was issued, so its completion covers that PV.
         tmem_stn<KW / 2>(T_P + bb * 64 + lane_off + (KW / 2) * hg, pk);
         float a0, a1, a2, a3;
         f2unpack(acc0, a0, a1);
