@@ -649,7 +649,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     constexpr int KW = kBN / NG;        // keys per group and tile
     constexpr int HD = D / NG;          // O columns per group
     constexpr int OC = HD < 32 ? HD : 32;
-    constexpr int NPOLY = (KW * 3) / 8; // keys per group whose 2^x runs on the FMA pipes
     const int hg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
@@ -768,7 +767,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const uint64_t dd = fadd2(f2pack(x[c], x[c + 1]), nm2);
           float d0, d1;
           f2unpack(dd, d0, d1);
-          if (c < NPOLY) {
+          // 3 of every 8 pairs on the FMA pipes, interleaved with the rest on
+          // the transcendental unit so that both pipes work at once
+          if (((c >> 1) & 7) < 3) {
             exp2_poly2(d0, d1, p0, p1);
           } else {
             p0 = ex2(d0);
