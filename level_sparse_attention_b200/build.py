@@ -9,7 +9,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["pyramid.cu", "mask.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu",
+SOURCES = ["pyramid.cu", "mask.cu", "score_tc.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu",
            "psa_noalloc.cu"]
 LIB = os.path.join(HERE, "libpsa.so")
 
@@ -23,8 +23,8 @@ def nvcc() -> str:
 
 def build(verbose: bool = False) -> str:
     srcs = [os.path.join(HERE, "csrc", s) for s in SOURCES]
-    deps = srcs + [os.path.join(HERE, "csrc", "psa_internal.cuh"),
-                   os.path.join(ROOT, "include", "psa.h")]
+    deps = srcs + [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))
+                   if f.endswith(".cuh")] + [os.path.join(ROOT, "include", "psa.h")]
     if os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps):
         return LIB
     tmp = LIB + ".tmp"

@@ -13,11 +13,10 @@
 // block ranked r takes the smallest level l with C_r < tau_l, C_r the mass of
 // the blocks ranked before it, else it is pruned.
 //
-// Three launches:
+// Three launches (the block logits themselves are in score_tc.cu):
 //   qmean_kernel   one CTA per query block; streams Q once (HBM-bound).
-//   score_kernel   register-tiled fp32 GEMM of query-block means against the
-//                  level-3 keys, logsumexp over each KV block's keys fused
-//                  into the epilogue.
+//   score_tc_kernel  split-precision tensor-core GEMM of query-block means
+//                  against the level-3 keys, logsumexp per KV block fused.
 //   assign_kernel  one warp per query block: softmax, bitonic sort of packed
 //                  (P, index) keys (in registers up to 1024 blocks, else in
 //                  shared memory), scan, cut, overrides, and the work list
@@ -78,123 +77,6 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
 }
 
 // -------------------------------------------------------------- scoring
-
-constexpr int kSgM = 64;       // query blocks per CTA tile
-constexpr int kSgN = 128;      // level-3 keys per CTA tile (16 KV blocks of 8 keys)
-constexpr int kSgK = 16;       // head-dim slice per stage
-constexpr int kSgPad = 4;      // row padding of the transposed shared tiles
-
-// Block logits as a register-tiled fp32 GEMM, C = q_bar [Nq x d] . K3 [rows3 x d]^T
-// per head, with the logsumexp over each KV block's 8 level-3 keys fused into
-// the epilogue.  256 threads; thread (tm, tn) owns 4 query blocks x the 8 keys
-// of one KV block, so its 32 accumulators give 4 block logits directly.
-// Operands are staged transposed in shared memory ([k][m], [k][n]),
-// double-buffered through registers: per k-step a thread reads 3 x 16 bytes
-// and issues 32 FMA.
-template <int D>
-__global__ void __launch_bounds__(256, 3) score_kernel(MaskArgs a, int m_tiles, int n_tiles,
-                                                    const float* __restrict__ qmean,
-                                                    const float* __restrict__ k3f,
-                                                    float* __restrict__ zlog) {
-  __shared__ __align__(16) float As[2][kSgK][kSgM + kSgPad];
-  __shared__ __align__(16) float Bs[2][kSgK][kSgN + kSgPad];
-  int id = blockIdx.x;
-  const int nt = id % n_tiles; id /= n_tiles;
-  const int mt = id % m_tiles;
-  const int bhq = id / m_tiles;
-  const int b = bhq / a.Hq, hq = bhq % a.Hq;
-  const int bhk = b * a.Hkv + hq / (a.Hq / a.Hkv);
-  const long long rows3 = ((long long)a.N + 7) / 8;
-  const int m0 = mt * kSgM;
-  const long long n0 = (long long)nt * kSgN;
-  const float* Ag = qmean + (long long)bhq * a.Nq * D;
-  const float* Bg = k3f + (long long)bhk * rows3 * D;
-  const int tid = threadIdx.x;
-  // a warp covers 8 query-block groups x 4 KV blocks, so each k-step reads
-  // 128 + 128 bytes of shared memory per warp for its 32 FMA per thread
-  const int lane = tid & 31, wid = tid >> 5;
-  const int tm = (wid >> 2) * 8 + (lane >> 2), tn = (wid & 3) * 4 + (lane & 3);
-
-  // global -> register staging: A 64x16 (one float4 per thread), B 128x16
-  // (two).  Consecutive threads take consecutive rows, so the transposed
-  // shared-memory stores of a warp hit 32 different banks.
-  const int ar = tid & 63, ak = (tid >> 6) * 4;
-  const int br0 = tid & 127, br1 = br0, bk = (tid >> 7) * 4;
-  float4 ra, rb0, rb1;
-  auto load = [&](int k0) {
-    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-    ra = (m0 + ar < a.Nq) ? *reinterpret_cast<const float4*>(Ag + (long long)(m0 + ar) * D + k0 + ak) : zero;
-    rb0 = (n0 + br0 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br0) * D + k0 + bk)) : zero;
-    rb1 = (n0 + br1 < rows3) ? __ldg(reinterpret_cast<const float4*>(Bg + (n0 + br1) * D + k0 + bk + 8)) : zero;
-  };
-  auto store = [&](int buf) {
-    As[buf][ak + 0][ar] = ra.x; As[buf][ak + 1][ar] = ra.y;
-    As[buf][ak + 2][ar] = ra.z; As[buf][ak + 3][ar] = ra.w;
-    Bs[buf][bk + 0][br0] = rb0.x; Bs[buf][bk + 1][br0] = rb0.y;
-    Bs[buf][bk + 2][br0] = rb0.z; Bs[buf][bk + 3][br0] = rb0.w;
-    Bs[buf][bk + 8][br1] = rb1.x; Bs[buf][bk + 9][br1] = rb1.y;
-    Bs[buf][bk + 10][br1] = rb1.z; Bs[buf][bk + 11][br1] = rb1.w;
-  };
-
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-
-  load(0);
-  store(0);
-  __syncthreads();
-  constexpr int NK = D / kSgK;
-#pragma unroll 1
-  for (int kt = 0; kt < NK; ++kt) {
-    const int buf = kt & 1;
-    if (kt + 1 < NK) load((kt + 1) * kSgK);
-#pragma unroll
-    for (int k = 0; k < kSgK; ++k) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[buf][k][tm * 4]);
-      const float4 bv0 = *reinterpret_cast<const float4*>(&Bs[buf][k][tn * 8]);
-      const float4 bv1 = *reinterpret_cast<const float4*>(&Bs[buf][k][tn * 8 + 4]);
-      const float am[4] = {av.x, av.y, av.z, av.w};
-      const float bn[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(am[i], bn[c], acc[i][c]);
-    }
-    if (kt + 1 < NK) {
-      store(buf ^ 1);
-      __syncthreads();
-    }
-  }
-
-  // epilogue: block logit = logsumexp over the KV block's level-3 keys
-  const long long j = n0 / 8 + tn;
-  if (j >= a.Nk) return;
-  const long long g0 = j * 8;
-  float lnc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const long long g = g0 + c;
-    lnc[c] = g < rows3 ? logf((float)min(8LL, (long long)a.N - g * 8)) : -INFINITY;
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int qa = m0 + tm * 4 + i;
-    if (qa >= a.Nq) continue;
-    float lg[8], mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      lg[c] = lnc[c] == -INFINITY ? -INFINITY : a.scale * acc[i][c] + lnc[c];
-      mx = fmaxf(mx, lg[c]);
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (lg[c] != -INFINITY) s += expf(lg[c] - mx);
-    zlog[((long long)bhq * a.Nq + qa) * a.Nk + j] = mx + logf(s);
-  }
-}
 
 // ------------------------------------------------------------ assignment
 //
@@ -436,23 +318,6 @@ cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, 
     qmean_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, (const __nv_bfloat16*)Q, qm);
   else
     qmean_kernel<float><<<grid, 256, 0, st>>>(a, (const float*)Q, qm);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, char* ws,
-                         cudaStream_t st) {
-  const MaskArgs a = make_mask_args(p, L, scale);
-  const int m_tiles = (L.Nq + kSgM - 1) / kSgM;
-  const int n_tiles = (int)((L.rows[3] + kSgN - 1) / kSgN);
-  const long long grid = (long long)p.B * p.Hq * m_tiles * n_tiles;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const float* qm = (const float*)(ws + L.qmean);
-  const float* k3 = (const float*)(ws + L.k3f);
-  float* z = (float*)(ws + L.zlog);
-  if (p.d == 128)
-    score_kernel<128><<<(unsigned)grid, 256, 0, st>>>(a, m_tiles, n_tiles, qm, k3, z);
-  else
-    score_kernel<64><<<(unsigned)grid, 256, 0, st>>>(a, m_tiles, n_tiles, qm, k3, z);
   return cudaGetLastError();
 }
 
