@@ -26,7 +26,8 @@
 //              exchanged per tile, P written back to TMEM as bf16, lazy O
 //              rescale (only when the running max grows by more than 2^8),
 //              epilogue O / lse split by column halves.
-// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,384+d).
+// TMEM columns: S0 [0,128) S1 [128,256) (P(t) over S(t)), O [256,256+d),
+// Q [384,384+d/2): QK^T reads Q from TMEM, so shared memory only feeds K and V.
 // Every mbarrier wait is bounded: on expiry the kernel records a timeout in
 // the workspace error word and winds down without trapping.
 #include "psa_internal.cuh"
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
-    mbar_init(bar(B_QEMPTY), 1);
+    mbar_init(bar(B_QEMPTY), 128 * kSoftGroups);   // Q copied to TMEM (smem Q free)
     for (int s = 0; s < KS; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
     for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 4 * kSoftGroups); }
@@ -252,7 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t T_S = tmem, T_P = tmem + 256, T_O = tmem + 384;
+  // TMEM columns: S0 [0,128) S1 [128,256) (P(t) is written over S(t), as bf16
+  // pairs, once both softmax groups have read it), O [256, 256+D), Q [384, 384+D/2)
+  const uint32_t T_S = tmem, T_O = tmem + 256, T_Q = tmem + 384;
 
   if (warp == 0) {
     // ---------------------------------------------------- K / Q producer
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int i = lane; i < n_ent; i += 32) lcache[i] = __ldg(lrow + i);
       __syncwarp();
       TileEntry cur = tile_entry(w, lrow, lcache, 0, lane);
-      if (iq > 0 && !warp_wait(bar(B_QEMPTY), (iq - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      if (iq > 0 && !warp_wait(bar(B_QEMPTY), (iq - 1) & 1, abort_flag, p.err)) { ok = false; break; }   // smem Q free
       if (lane == 0) {
         mbar_expect_tx(bar(B_QFULL), C::Q_BYTES);
         for (int h = 0; h < C::HALVES; ++h)
@@ -391,8 +394,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_bf16(kBM, kBN, false);
       constexpr uint32_t ID_PV = idesc_bf16(kBM, D, true);
-      static_assert(kBM * 128 == C::HALF, "Q and K tiles share one half-tile layout");
-      const uint64_t qdesc0 = sdesc(sbase + C::OFF_Q, 16, 1024);
       const uint64_t kdesc0 = sdesc(sbase + C::OFF_K, 16, 1024);
       const uint64_t vdesc0 = sdesc(sbase + C::OFF_V, C::HALF, 1024);
       bool ok = true;
@@ -402,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (!wait_bar(bar(B_VFULL + s), (u / VS) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
         const uint64_t vd = vdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
-        const uint32_t dP = T_P + bb * 64;
+        const uint32_t dP = T_S + bb * 128;          // P(u) written over S(u)
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k)
           mma_ts(T_O, dP + k * 8, vd + (uint64_t)(k * (2048 >> 4)), ID_PV,
@@ -423,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint32_t dS = T_S + bb * 128;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          constexpr uint32_t kHalfStep = C::HALF >> 4;   // same layout for Q and K halves
+          constexpr uint32_t kHalfStep = C::HALF >> 4;
           const uint64_t off = (uint64_t)((k >> 2) * kHalfStep + (k & 3) * 2);
-          mma_ss(dS, qdesc0 + off, kd + off, ID_QK, k > 0 ? 1u : 0u);
+          mma_ts(dS, T_Q + k * 8, kd + off, ID_QK, k > 0 ? 1u : 0u);   // A = Q in TMEM
         }
         mma_commit(bar(B_SFULL + bb));
         mma_commit(bar(B_KEMPTY + s));
@@ -438,11 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
-        if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!wait_bar(bar(B_QEMPTY), iq & 1, abort_flag, p.err)) { ok = false; break; }   // Q in TMEM
         ++iq;
         for (int t = 0; ok && t < T; ++t) {
           ok = issue_qk(g + t);
-          if (ok && t == T - 1) mma_commit(bar(B_QEMPTY));
           if (ok && t >= 1) ok = issue_pv(g + t - 1, t == 1);
         }
         if (ok) ok = issue_pv(g + T - 1, T == 1);
@@ -484,13 +484,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int i = 0; i < NG; ++i) all[i] = buf[i * 128 + r];
     };
     const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-    int g = 0;
+    int g = 0, iqs = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int qpos = qa * kBM + r;
       float m = -INFINITY, lsum = 0.f;
+      if (T > 0) {
+        // Q of this query block into TMEM (the A operand of QK^T): row r,
+        // packed bf16 pairs [hg*D/4, (hg+1)*D/4) of the row, read out of the
+        // 128-byte-swizzled TMA tile.  The previous block's QK^T are complete
+        // (its last PV, which followed them, was waited for in the epilogue).
+        ok = ok && warp_wait(bar(B_QFULL), iqs & 1, abort_flag, p.err);
+        if (ok) {
+          constexpr int QW = D / 2 / NG;               // packed columns per group
+          uint32_t qv[QW];
+#pragma unroll
+          for (int c = 0; c < QW; c += 4) {
+            const int e = 2 * (hg * QW + c);             // first element of this 16-byte chunk
+            const int h = e >> 6, ch = (e & 63) >> 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                smem + C::OFF_Q + h * (kBM * 128) + r * 128 + ((ch ^ (r & 7)) << 4));
+            qv[c] = v.x; qv[c + 1] = v.y; qv[c + 2] = v.z; qv[c + 3] = v.w;
+          }
+          tmem_stn<QW>(T_Q + lane_off + hg * QW, qv);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_QEMPTY));
+        ++iqs;
+      }
       for (int t = 0; t < T; ++t) {
         const int gt = g + t, bb = gt & 1, ms = gt % MS;
         ok = ok && warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) &&
@@ -601,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         // P(gt - 2) in this buffer has been consumed: S(gt) was committed after
         // PV(gt - 2) was issued, so its completion covers that PV.
-        tmem_stn<KW / 2>(T_P + bb * 64 + lane_off + (KW / 2) * hg, pk);
+        tmem_stn<KW / 2>(T_S + bb * 128 + lane_off + (KW / 2) * hg, pk);   // P over S
         float a0, a1, a2, a3;
         f2unpack(acc0, a0, a1);
         f2unpack(acc1, a2, a3);
