@@ -58,6 +58,53 @@ def peaks():
         return 1590.0, 6650.0, "fallback"
 
 
+# --------------------------------------------------------- multi-rank plumbing
+#
+# Every (batch, head) problem of the forward pass is independent, so N ranks
+# each run their own batch of the workload's shape with no data-path
+# collective (weak scaling).  The only collectives are measurement: a barrier
+# around the timed region and a max over ranks of the timed milliseconds.
+
+def rank_batch0(rank: int, B: int) -> int:
+    """Global index of the first batch element that `rank` runs: rank r runs
+    elements [r*B, (r+1)*B) of a global batch of world*B."""
+    return rank * B
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of `x` over all ranks (x itself when world == 1)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Throughput of the whole job: the work all ranks did over the slowest
+    rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
+def mask_bytes(w: W.Workload) -> float:
+    """Algorithmic HBM bytes of the mask stage: Q read once, the fp32 level-3
+    keys read once per KV head, the int8 level map written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    return float(w.B * w.Hq * w.N * w.d * es + w.B * w.Hkv * (-(-w.N // 8)) * w.d * 4
+                 + w.B * w.Hq * w.Nq * w.Nk)
+
+
+def pyramid_bytes(w: W.Workload) -> float:
+    """Algorithmic HBM bytes of the pyramid stage: K and V read once, levels
+    1..3 of both written once (1/2 + 1/4 + 1/8 of the input), the fp32
+    level-3 keys written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    return float(2 * w.B * w.Hkv * w.N * w.d * es * (1 + 0.875)
+                 + w.B * w.Hkv * (-(-w.N // 8)) * w.d * 4)
+
+
 # ------------------------------------------------------------- CPU oracle leg
 
 def cpu_sample(w: W.Workload, n_heads: int):
@@ -168,7 +215,7 @@ def run_ours(args, rank, world, local_rank):
     p = P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk, tau, w.causal,
                       w.forced_prefix_tokens, 0.0,
                       torch.bfloat16 if w.dtype == "bf16" else torch.float32)
-    inp = W.make_inputs(w)
+    inp = W.make_inputs(w, batch0=rank_batch0(rank, w.B))
 
     def host(x):
         t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
@@ -227,13 +274,8 @@ def run_ours(args, rank, world, local_rank):
     pyr_ms = [e[0].elapsed_time(e[1]) for e in ev]
     mask_ms = [e[1].elapsed_time(e[2]) for e in ev]
     attn_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    tot_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms = float(t.item())
-    ms = tot_ms / args.steps
-    value = dense * world / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(sum(step_ms), world, dev) / args.steps
+    value = whole_job_tflops(dense, world, ms)
 
     # end to end through the public API with host buffers: H2D of Q, K, V, the
     # forward, D2H of O, every step inside the timed region
@@ -250,18 +292,17 @@ def run_ours(args, rank, world, local_rank):
         hout.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     P.check_device(p, ws)
 
     bf16_peak, hbm_peak, peak_kind = peaks()
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = executed / (attn_avg * 1e-3) / 1e12
     es = 2 if w.dtype == "bf16" else 4
-    pyr_bytes = 2 * w.B * w.Hkv * w.N * w.d * es * (1 + 0.875) + w.B * w.Hkv * (-(-w.N // 8)) * w.d * 4
+    pyr_avg = sum(pyr_ms) / len(pyr_ms)
+    mask_avg = sum(mask_ms) / len(mask_ms)
+    pyr_gbs = pyramid_bytes(w) / (pyr_avg * 1e-3) / 1e9
+    mask_gbs = mask_bytes(w) / (mask_avg * 1e-3) / 1e9
     if rank != 0:
         return
     cpu = None
@@ -274,16 +315,17 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded smooth 3-D field + noise)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+        "config": {"workload": w.name, "global_batch": w.B * world, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                    "q_blk": w.q_blk, "kv_blk": w.kv_blk, "tau": [round(t, 6) for t in tau],
                    "causal": w.causal, "skipped_dense_fraction": 1.0 - executed / dense,
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": f"independent batch per GPU x{world}"},
         "ms_per_call": ms, "pct_bf16_peak_dense_equiv": 100.0 * value / world / bf16_peak,
         "executed_tflops": executed * world / (ms * 1e-3) / 1e12,
-        "kernel_ms": {"pyramid": sum(pyr_ms) / len(pyr_ms), "mask": sum(mask_ms) / len(mask_ms),
-                      "attention": attn_avg},
-        "pyramid_gbs": pyr_bytes / (sum(pyr_ms) / len(pyr_ms) * 1e-3) / 1e9,
+        "kernel_ms": {"pyramid": pyr_avg, "mask": mask_avg, "attention": attn_avg},
+        "hbm": {"peak_gbs": hbm_peak, "peak_kind": f"{peak_kind} copy",
+                "pyramid": {"bytes": pyramid_bytes(w), "gbs": pyr_gbs, "frac": pyr_gbs / hbm_peak},
+                "mask": {"bytes": mask_bytes(w), "gbs": mask_gbs, "frac": mask_gbs / hbm_peak}},
         "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": bf16_peak, "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s",
                      "frac": achieved / bf16_peak, "traffic": None,

@@ -138,6 +138,12 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// How many of every 8 exponential pairs of a softmax tile take the FMA-pipe
+// polynomial above.  With one 128-row query tile per CTA the tensor-core
+// chain, not the transcendental unit, limits a tile (3 of 8 measured 2%
+// slower than 0 on the 1.3B video shape), so all go to the MUFU.
+constexpr int kPolyPairs = 0;
+
 // ------------------------------------------------------------ work list
 
 // Per query block: entry counts per level give where each level starts in
@@ -610,9 +616,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const uint64_t dd = fadd2(f2pack(x[c], x[c + 1]), nm2);
           float d0, d1;
           f2unpack(dd, d0, d1);
-          // 3 of every 8 pairs on the FMA pipes, interleaved with the rest on
-          // the transcendental unit so that both pipes work at once
-          if (((c >> 1) & 7) < 3) {
+          // kPolyPairs of every 8 pairs on the FMA pipes, interleaved with
+          // the rest on the transcendental unit
+          if (((c >> 1) & 7) < kPolyPairs) {
             exp2_poly2(d0, d1, p0, p1);
           } else {
             p0 = ex2(d0);

@@ -195,9 +195,12 @@ class Inputs:
 
 
 def make_inputs(w: Workload, heads_q: Optional[List[int]] = None,
-                heads_kv: Optional[List[int]] = None) -> Inputs:
+                heads_kv: Optional[List[int]] = None, batch0: int = 0) -> Inputs:
     """Generate the workload's inputs.  ``heads_q``/``heads_kv`` restrict the
-    heads generated (others are left zero) so that samples stay cheap."""
+    heads generated (others are left zero) so that samples stay cheap.
+    ``batch0`` is the global index of the first batch element: local element b
+    holds global batch element batch0 + b, so that ranks that each run their
+    own share of a larger batch see different data."""
     N, d = w.N, w.d
     store = np.uint16 if w.dtype == "bf16" else np.float32
     out = []
@@ -205,7 +208,7 @@ def make_inputs(w: Workload, heads_q: Optional[List[int]] = None,
         arr = np.zeros((w.B, H, N, d), dtype=store)
         for b in range(w.B):
             for h in (range(H) if sel is None else sel):
-                vals = head_values(w, ti, h, b)
+                vals = head_values(w, ti, h, batch0 + b)
                 arr[b, h] = f32_to_bf16_bits(vals) if w.dtype == "bf16" else vals
         out.append(arr)
     return Inputs(w, *out)
