@@ -49,6 +49,26 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# attention launch, from an ncu capture, keyed by the workload and a hash of
+# the attention kernel's sources.  A kernel that has changed since the
+# counters were taken has no entry, and the roofline's traffic is then null.
+# The Wan2.1-1.3B figure is a 6-head capture (278.1 MB) scaled by 2 to the
+# 12-head launch: every head reads its own Q, K and V levels once, so the
+# traffic grows in proportion to the heads.
+ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh")
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "c6b363e67eeee4ae"): 2 * (236.379136e6 + 41.732096e6)}
+
+
+def attn_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "level_sparse_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -328,7 +348,8 @@ def run_ours(args, rank, world, local_rank):
                 "mask": {"bytes": mask_bytes(w), "gbs": mask_gbs, "frac": mask_gbs / hbm_peak}},
         "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": bf16_peak, "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s",
-                     "frac": achieved / bf16_peak, "traffic": None,
+                     "frac": achieved / bf16_peak,
+                     "traffic": ATTN_TRAFFIC.get((w.name, w.Hq, attn_source_hash())),
                      "executed_flops_per_launch": executed,
                      "padding_fraction": 1.0 - (keys_per_row.sum() / max(padded_keys, 1.0))},
         "cpu_baseline": cpu,
