@@ -192,9 +192,13 @@ def workspace_layout(p: Params) -> dict:
         n = a256(p.B * p.Hkv * rows[l] * p.d * es)
         L["kp"][l], off = off, off + n
         L["vp"][l], off = off, off + n
-    L["k3f"], off = off, off + a256(p.B * p.Hkv * rows[3] * p.d * 4)
+    # fp32 GEMM operands as tf32 head + exact tail pairs
+    k3 = a256(p.B * p.Hkv * rows[3] * p.d * 4)
+    L["k3h"], off = off, off + k3
+    L["k3l"], off = off, off + k3
     rq = p.B * p.Hq * Nq
-    L["qmean"], off = off, off + a256(rq * p.d * 4)
+    L["qmh"], off = off, off + a256(rq * p.d * 4)
+    L["qml"], off = off, off + a256(rq * p.d * 4)
     L["zlog"], off = off, off + a256(rq * Nk * 4)
     L["map"], off = off, off + a256(rq * Nk)
     L["counts"], off = off, off + a256(rq * 16)

@@ -28,51 +28,94 @@ namespace {
 
 // -------------------------------------------------------------- q means
 
+// One CTA of 256 threads per query block.  Thread t takes the 8-column chunk
+// t % (d/8) of rows t / (d/8) + k * 256/(d/8) (at most 8 rows: q_blk <= 128,
+// d >= 64) and issues all its loads before adding.  Lanes holding the same
+// chunk are summed with shuffles, the 8 warps' partial sums in shared memory.
+template <typename T> struct QVec;
+template <> struct QVec<__nv_bfloat16> {
+  uint4 raw;
+  __device__ void load(const __nv_bfloat16* p) { raw = *reinterpret_cast<const uint4*>(p); }
+  __device__ void add_to(float* acc) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __bfloat1622float2(h[i]);
+      acc[2 * i] += v.x;
+      acc[2 * i + 1] += v.y;
+    }
+  }
+};
+template <> struct QVec<float> {
+  float4 u, w;
+  __device__ void load(const float* p) {
+    u = reinterpret_cast<const float4*>(p)[0];
+    w = reinterpret_cast<const float4*>(p)[1];
+  }
+  __device__ void add_to(float* acc) const {
+    acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
+    acc[4] += w.x; acc[5] += w.y; acc[6] += w.z; acc[7] += w.w;
+  }
+};
+
 template <typename T>
 __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restrict__ Q,
-                                                    float* __restrict__ qmean) {
+                                                    float* __restrict__ qmh,
+                                                    float* __restrict__ qml) {
   const int row = blockIdx.x;               // (b*Hq + h) * Nq + qa
   const int qa = row % a.Nq;
   const long long bh = row / a.Nq;
   const int lo = qa * a.q_blk;
   const int n = min(a.q_blk, a.N - lo);
-  const int chunks = a.d / 8;
-  const int parts = blockDim.x / chunks;    // row slices summed by separate threads
+  const int chunks = a.d / 8;               // 16 or 8
+  const int parts = 256 / chunks;           // rows read side by side: 16 or 32
   const int c = threadIdx.x % chunks;
   const int part = threadIdx.x / chunks;
+  const T* base = Q + (bh * a.N + lo) * a.d + c * 8;
+  QVec<T> raw[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = part + k * parts;
+    if (r < n) raw[k].load(base + (long long)r * a.d);
+  }
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  const T* base = Q + (bh * a.N + lo) * a.d + c * 8;
-  for (int r = part; r < n; r += parts) {
-    const T* src = base + (long long)r * a.d;
-    if constexpr (sizeof(T) == 2) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(src);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 v = __bfloat1622float2(h[i]);
-        acc[2 * i] += v.x;
-        acc[2 * i + 1] += v.y;
-      }
-    } else {
-      const float4 u = reinterpret_cast<const float4*>(src)[0];
-      const float4 w = reinterpret_cast<const float4*>(src)[1];
-      acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
-      acc[4] += w.x; acc[5] += w.y; acc[6] += w.z; acc[7] += w.w;
-    }
-  }
-  __shared__ float red[256 * 8];
+  for (int k = 0; k < 8; ++k)
+    if (part + k * parts < n) raw[k].add_to(acc);
+  // lanes l, l + chunks, ... of a warp hold the same chunk
+  for (int o = chunks; o < 32; o <<= 1)
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[threadIdx.x * 8 + e] = acc[e];
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  __shared__ float red[8][16][8];           // [warp][chunk][column]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < chunks)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[warp][lane][e] = acc[e];
   __syncthreads();
-  if (part == 0) {
-    for (int q = 1; q < parts; ++q)
+  if (threadIdx.x < chunks) {
+    float sum[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += red[(q * chunks + c) * 8 + e];
-    float* dst = qmean + (long long)row * a.d + c * 8;
+    for (int e = 0; e < 8; ++e) sum[e] = red[0][c][e];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = __fdiv_rn(acc[e], (float)n);
+    for (int w = 1; w < 8; ++w)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sum[e] += red[w][c][e];
+    // the mean in fp32, stored as tf32 head + exact tail
+    float hd[8], tl[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float m = __fdiv_rn(sum[e], (float)n);
+      hd[e] = tf32_head(m);
+      tl[e] = m - hd[e];
+    }
+    float4* dh = reinterpret_cast<float4*>(qmh + (long long)row * a.d + c * 8);
+    float4* dl = reinterpret_cast<float4*>(qml + (long long)row * a.d + c * 8);
+    dh[0] = make_float4(hd[0], hd[1], hd[2], hd[3]);
+    dh[1] = make_float4(hd[4], hd[5], hd[6], hd[7]);
+    dl[0] = make_float4(tl[0], tl[1], tl[2], tl[3]);
+    dl[1] = make_float4(tl[4], tl[5], tl[6], tl[7]);
   }
 }
 
@@ -313,11 +356,12 @@ cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, 
                          cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, 0.f);
   const int grid = p.B * p.Hq * L.Nq;
-  float* qm = (float*)(ws + L.qmean);
+  float* qh = (float*)(ws + L.qmh);
+  float* ql = (float*)(ws + L.qml);
   if (p.dtype == PSA_BF16)
-    qmean_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, (const __nv_bfloat16*)Q, qm);
+    qmean_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, (const __nv_bfloat16*)Q, qh, ql);
   else
-    qmean_kernel<float><<<grid, 256, 0, st>>>(a, (const float*)Q, qm);
+    qmean_kernel<float><<<grid, 256, 0, st>>>(a, (const float*)Q, qh, ql);
   return cudaGetLastError();
 }
 

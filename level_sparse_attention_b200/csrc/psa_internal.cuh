@@ -23,8 +23,10 @@ struct Layout {
   size_t err;                 // int32 device error word (+ padding)
   size_t kp[kLevels];         // pooled keys, level 1..3 (index 0 unused)
   size_t vp[kLevels];         // pooled values, level 1..3
-  size_t k3f;                 // level-3 keys in fp32 [B, Hkv, ceil(N/8), d]
-  size_t qmean;               // query-block means fp32 [B, Hq, Nq, d]
+  // fp32 operands of the block-logit GEMM, each split into a tf32 head (low
+  // 13 mantissa bits clear) and the exact remainder: x = head + tail
+  size_t k3h, k3l;            // level-3 keys [B, Hkv, ceil(N/8), d]
+  size_t qmh, qml;            // query-block means [B, Hq, Nq, d]
   size_t zlog;                // block logits fp32 [B, Hq, Nq, Nk]
   size_t map;                 // internal level map int8 [B, Hq, Nq, Nk]
   size_t counts;              // int4 per query block: entries at level 0..3
@@ -49,9 +51,12 @@ inline __host__ __device__ Layout make_layout(const psa_params_t& p) {
     L.kp[l] = off; off += bytes;
     L.vp[l] = off; off += bytes;
   }
-  L.k3f = off; off += align256((size_t)p.B * p.Hkv * L.rows[3] * p.d * 4);
+  const size_t k3_bytes = align256((size_t)p.B * p.Hkv * L.rows[3] * p.d * 4);
+  L.k3h = off; off += k3_bytes;
+  L.k3l = off; off += k3_bytes;
   const size_t rowsq = (size_t)p.B * p.Hq * L.Nq;
-  L.qmean = off; off += align256(rowsq * p.d * 4);
+  L.qmh = off; off += align256(rowsq * p.d * 4);
+  L.qml = off; off += align256(rowsq * p.d * 4);
   L.zlog = off; off += align256(rowsq * L.Nk * 4);
   L.map = off; off += align256(rowsq * L.Nk);
   L.counts = off; off += align256(rowsq * 16);
@@ -87,6 +92,11 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// tf32 head of x (low 13 mantissa bits cleared) and the exact remainder.
+__device__ __forceinline__ float tf32_head(float x) {
+  return __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

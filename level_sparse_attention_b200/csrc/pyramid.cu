@@ -1,5 +1,6 @@
 // Pyramid KV construction: average pooling of K and V into levels 1..3
-// (2x, 4x, 8x), plus the level-3 keys in fp32 for block scoring.
+// (2x, 4x, 8x), plus the level-3 keys in fp32 for block scoring, stored as a
+// tf32 head and the exact remainder (the split operands of the scoring GEMM).
 //
 // Method: top168.com article on PSA (arXiv:2512.04025), pyramid paragraph and
 // component one — the bottom level is the original KV and each level above is
@@ -69,7 +70,7 @@ template <> struct PyrOcc<float> { static constexpr int kMinBlocks = 2; };
 // every mean a multiplication; otherwise counts come from `valid`.
 template <bool FULL, typename T>
 __device__ __forceinline__ void pool_group(const Vec4<T>* raw, int valid, T* p1, T* p2, T* p3,
-                                           float* pf, int d) {
+                                           float* pf, float* pl, int d) {
   // rows are consumed pairwise: each level-1 row is stored as soon as its
   // two tokens are summed, each level-2 row as soon as its two level-1 sums
   // are, so that few sums are live at once
@@ -113,7 +114,16 @@ __device__ __forceinline__ void pool_group(const Vec4<T>* raw, int valid, T* p1,
 #pragma unroll
   for (int e = 0; e < 4; ++e) m[e] = FULL ? s3[e] * 0.125f : mean_of(s3[e], valid);
   Vec4<T>::store(p3, m);
-  if (pf) Vec4<float>::store(pf, m);
+  if (pf) {                           // level-3 key in fp32 as tf32 head + exact tail
+    float h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      h[e] = tf32_head(m[e]);
+      l[e] = m[e] - h[e];
+    }
+    Vec4<float>::store(pf, h);
+    Vec4<float>::store(pl, l);
+  }
 }
 
 // grid: x = (groups << chunk_shift) / 256 rounded up, y = KV heads of all
@@ -121,7 +131,7 @@ __device__ __forceinline__ void pool_group(const Vec4<T>* raw, int valid, T* p1,
 template <typename T>
 __global__ void __launch_bounds__(256, PyrOcc<T>::kMinBlocks)
 pyramid_kernel(PyrArgs a, const T* __restrict__ K, const T* __restrict__ V, T* kp1, T* kp2,
-               T* kp3, T* vp1, T* vp2, T* vp3, float* k3f) {
+               T* kp3, T* vp1, T* vp2, T* vp3, float* k3h, float* k3l) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (a.groups << a.chunk_shift)) return;
   const int c = i & ((1 << a.chunk_shift) - 1);
@@ -138,18 +148,20 @@ pyramid_kernel(PyrArgs a, const T* __restrict__ K, const T* __restrict__ V, T* k
     T* p1 = d1 + ((size_t)bh * a.rows1 + (size_t)g * 4) * a.d + c * 4;
     T* p2 = d2 + ((size_t)bh * a.rows2 + (size_t)g * 2) * a.d + c * 4;
     T* p3 = d3 + ((size_t)bh * a.rows3 + g) * a.d + c * 4;
-    float* pf = is_v ? nullptr : k3f + ((size_t)bh * a.rows3 + g) * a.d + c * 4;
+    const size_t o3 = ((size_t)bh * a.rows3 + g) * a.d + c * 4;
+    float* pf = is_v ? nullptr : k3h + o3;
+    float* pl = is_v ? nullptr : k3l + o3;
     // all loads first, so that 8 are in flight per thread
     Vec4<T> raw[8];
     if (valid == 8) {
 #pragma unroll
       for (int r = 0; r < 8; ++r) raw[r].load(src + (size_t)r * a.d);
-      pool_group<true>(raw, 8, p1, p2, p3, pf, a.d);
+      pool_group<true>(raw, 8, p1, p2, p3, pf, pl, a.d);
     } else {
 #pragma unroll
       for (int r = 0; r < 8; ++r)
         if (r < valid) raw[r].load(src + (size_t)r * a.d);
-      pool_group<false>(raw, valid, p1, p2, p3, pf, a.d);
+      pool_group<false>(raw, valid, p1, p2, p3, pf, pl, a.d);
     }
   }
 }
@@ -174,12 +186,13 @@ cudaError_t launch_pyramid(const psa_params_t& p, const Layout& L, const void* K
     using T = __nv_bfloat16;
     pyramid_kernel<T><<<grid, block, 0, st>>>(
         a, (const T*)K, (const T*)V, (T*)(ws + L.kp[1]), (T*)(ws + L.kp[2]), (T*)(ws + L.kp[3]),
-        (T*)(ws + L.vp[1]), (T*)(ws + L.vp[2]), (T*)(ws + L.vp[3]), (float*)(ws + L.k3f));
+        (T*)(ws + L.vp[1]), (T*)(ws + L.vp[2]), (T*)(ws + L.vp[3]), (float*)(ws + L.k3h),
+        (float*)(ws + L.k3l));
   } else {
     pyramid_kernel<float><<<grid, block, 0, st>>>(
         a, (const float*)K, (const float*)V, (float*)(ws + L.kp[1]), (float*)(ws + L.kp[2]),
         (float*)(ws + L.kp[3]), (float*)(ws + L.vp[1]), (float*)(ws + L.vp[2]),
-        (float*)(ws + L.vp[3]), (float*)(ws + L.k3f));
+        (float*)(ws + L.vp[3]), (float*)(ws + L.k3h), (float*)(ws + L.k3l));
   }
   return cudaGetLastError();
 }

@@ -62,8 +62,28 @@ def test_pyramid_levels(name):
                 got = G.to_f64(run.view(key, shape, tdt, l)[0, hk])
                 tol = (2.0 ** -8 if w.dtype == "bf16" else 1e-6) * np.abs(ref) + 1e-6
                 assert np.all(np.abs(got - ref) <= tol), (key, l, np.abs(got - ref).max())
-        k3 = G.to_f64(run.view("k3f", (w.B, w.Hkv, L["rows"][3], w.d), torch.float32)[0, hk])
+        shape3 = (w.B, w.Hkv, L["rows"][3], w.d)
+        head = run.view("k3h", shape3, torch.float32)[0, hk]
+        tail = run.view("k3l", shape3, torch.float32)[0, hk]
+        # the head is a tf32 value (low 13 mantissa bits clear); head + tail is
+        # the fp32 level-3 key
+        assert int((head.view(torch.int32) & 0x1FFF).abs().max()) == 0
+        k3 = G.to_f64(head) + G.to_f64(tail)
         assert np.abs(k3 - pyr.keys[3]).max() <= 1e-5
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_query_block_means(name):
+    w, inp, ref, run = setup(name)
+    L = P.workspace_layout(run.p)
+    shape = (w.B, w.Hq, L["Nq"], w.d)
+    head = run.view("qmh", shape, torch.float32)
+    tail = run.view("qml", shape, torch.float32)
+    assert int((head.view(torch.int32) & 0x1FFF).abs().max()) == 0
+    qm = G.to_f64(head) + G.to_f64(tail)
+    for (b, h), _ in ref.items():
+        want = O.query_block_means(inp.as_f64("q", b, h), w.q_blk)
+        assert np.abs(qm[b, h] - want).max() <= 1e-5 * max(1.0, np.abs(want).max())
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
