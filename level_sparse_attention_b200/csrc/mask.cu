@@ -150,27 +150,53 @@ __device__ __forceinline__ T warp_excl_scan(T v, T* total) {
   return x - v;
 }
 
-// Writes the work list of one query block from its level row `lev` (shared):
-// KV block indices at level 0, then 1, 2, 3, each in increasing index order.
+// Writes the work list of one query block from its level row `lev` (shared,
+// padded with -1 up to a multiple of 16 bytes): KV block indices at level 0,
+// then 1, 2, 3, each in increasing index order.  Each lane owns a contiguous,
+// 16-byte aligned run of the row, read 16 levels at a time; byte-wise SIMD
+// compares count and locate each level, and two packed scans (two 16-bit
+// counts per word; a row has at most 8192 blocks) give every lane its
+// positions.
 __device__ void emit_list_warp(const int8_t* lev, int Nk, int* __restrict__ list_row,
                                int4* __restrict__ count_row) {
   const int lane = threadIdx.x & 31;
-  const int per = (Nk + 31) / 32;
+  const int per = (((Nk + 31) / 32) + 15) & ~15;
   const int j0 = lane * per, j1 = min(Nk, j0 + per);
-  int base = 0;
-  int cnt[kLevels];
+  int cnt[kLevels] = {0, 0, 0, 0};
+  for (int j = j0; j < j1; j += 16) {
+    const uint4 w = *reinterpret_cast<const uint4*>(lev + j);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int l = 0; l < kLevels; ++l) {
-    int mine = 0;
-    for (int j = j0; j < j1; ++j) mine += lev[j] == l;
-    int total;
-    int pos = base + warp_excl_scan(mine, &total);
-    for (int j = j0; j < j1; ++j)
-      if (lev[j] == l) list_row[pos++] = j;
-    cnt[l] = total;
-    base += total;
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int l = 0; l < kLevels; ++l) cnt[l] += __popc(__vcmpeq4(x[k], 0x01010101u * l)) >> 3;
   }
-  if (lane == 0) *count_row = make_int4(cnt[0], cnt[1], cnt[2], cnt[3]);
+  int t01, t23;
+  const int p01 = warp_excl_scan(cnt[0] | (cnt[1] << 16), &t01);
+  const int p23 = warp_excl_scan(cnt[2] | (cnt[3] << 16), &t23);
+  const int tot[kLevels] = {t01 & 0xffff, t01 >> 16, t23 & 0xffff, t23 >> 16};
+  int pos[kLevels];
+  pos[0] = p01 & 0xffff;
+  pos[1] = tot[0] + (p01 >> 16);
+  pos[2] = tot[0] + tot[1] + (p23 & 0xffff);
+  pos[3] = tot[0] + tot[1] + tot[2] + (p23 >> 16);
+  for (int j = j0; j < j1; j += 16) {
+    const uint4 w = *reinterpret_cast<const uint4*>(lev + j);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int l = 0; l < kLevels; ++l) {
+        uint32_t m = __vcmpeq4(x[k], 0x01010101u * l);   // 0xff in every matching byte
+        while (m) {
+          const int b = __ffs(m) - 1;                     // lowest bit of the lowest match
+          list_row[pos[l]++] = j + 4 * k + (b >> 3);
+          m &= ~(0xffu << (b & ~7));
+        }
+      }
+    }
+  }
+  if (lane == 0) *count_row = make_int4(tot[0], tot[1], tot[2], tot[3]);
 }
 
 // Bitonic sort of 32*K 64-bit keys held in registers, descending.  Element
@@ -214,6 +240,41 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[K]) {
   }
 }
 
+// Candidate set of the register path: at most kCand blocks, kCandPerLane
+// keys per lane.
+constexpr int kCandPerLane = 4;
+constexpr int kCand = 32 * kCandPerLane;
+
+__host__ __device__ inline size_t assign_key_bytes(int K, int n2) {
+  return K == 0 ? (size_t)n2 * 8 : (K > kCandPerLane ? (size_t)kCand * 8 : 0);
+}
+
+// Sorted keys (descending; lane L holds ranks L*K .. L*K + K - 1) -> levels of
+// the first n ranks: exclusive running mass c, level = first tau above c.
+template <int K>
+__device__ __forceinline__ void levels_from_sorted(const unsigned long long (&v)[K], int n,
+                                                   const float* tau, int8_t* lev) {
+  const int lane = threadIdx.x & 31;
+  float mine = 0.f;
+#pragma unroll
+  for (int r = 0; r < K; ++r)
+    if (lane * K + r < n) mine += __uint_as_float((unsigned)(v[r] >> 32));
+  float total;
+  float c = warp_excl_scan(mine, &total);
+#pragma unroll
+  for (int r = 0; r < K; ++r) {
+    if (lane * K + r < n) {
+      const int j = (int)(0xffffffffu - (unsigned)(v[r] & 0xffffffffu));
+      int l = -1;
+#pragma unroll
+      for (int t = kLevels - 1; t >= 0; --t)
+        if (c < tau[t]) l = t;
+      lev[j] = (int8_t)l;
+      c += __uint_as_float((unsigned)(v[r] >> 32));
+    }
+  }
+}
+
 template <int K>
 __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
                               const float* __restrict__ zlog, int8_t* __restrict__ map_ws,
@@ -224,7 +285,9 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   const int row = blockIdx.x * rows_per_cta + warp;
   if (row >= nrows) return;                 // whole warp; no block barriers below
   const int lev_stride = (a.Nk + 15) & ~15;
-  const size_t key_bytes = K > 0 ? 0 : (size_t)n2 * 8;       // keys in registers when K > 0
+  // keys in shared memory: all n2 of them for the shared-memory sort, the
+  // candidate set for the register path
+  const size_t key_bytes = assign_key_bytes(K, n2);
   unsigned long long* key = reinterpret_cast<unsigned long long*>(smem) + (size_t)warp * (key_bytes / 8);
   int8_t* lev = reinterpret_cast<int8_t*>(smem + (size_t)rows_per_cta * key_bytes) +
                 (size_t)warp * lev_stride;
@@ -247,34 +310,127 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
     const float pj = expf(z[i] - mx) * inv;
     return ((unsigned long long)__float_as_uint(pj) << 32) | (0xffffffffu - (unsigned)i);
   };
-  for (int j = lane; j < a.Nk; j += 32) lev[j] = -1;
+  for (int j = lane; j < lev_stride; j += 32) lev[j] = -1;
 
   // rank by P descending (ties to the lower index), exclusive running mass,
   // level = first tau the running mass is below
   if constexpr (K > 0) {
-    // sorted keys stay in registers: lane L holds ranks L*K .. L*K + K - 1
-    unsigned long long v[K > 0 ? K : 1];
-#pragma unroll
-    for (int r = 0; r < K; ++r) v[r] = make_key(lane * K + r);
-    warp_bitonic_desc<K>(v);
-    __syncwarp();                          // lev[] initialised by all lanes
-    float mine = 0.f;
-#pragma unroll
-    for (int r = 0; r < K; ++r)
-      if (lane * K + r < nvis) mine += __uint_as_float((unsigned)(v[r] >> 32));
-    float total;
-    float c = warp_excl_scan(mine, &total);
+    // P of element i = lane*K + r in register r (0 past the visible blocks)
+    float pj[K];
 #pragma unroll
     for (int r = 0; r < K; ++r) {
-      if (lane * K + r < nvis) {
-        const int j = (int)(0xffffffffu - (unsigned)(v[r] & 0xffffffffu));
-        int l = -1;
+      const int i = lane * K + r;
+      pj[r] = i < nvis ? expf(z[i] - mx) * inv : 0.f;
+    }
+    __syncwarp();                          // lev[] initialised by all lanes
+    bool done = false;
+    if constexpr (K > kCandPerLane) {
+      // Candidate cut: blocks with P >= t form a prefix of the ranking, and
+      // when their mass reaches tau_3 every block after them has a running
+      // mass >= tau_3, i.e. is pruned.  t is bisected until the candidates
+      // number at most kCand, with a margin of 1e-3 on the mass so that the
+      // rounding of this sum against the scan below cannot matter; then
+      // only the candidates are sorted.
+      const float target = a.tau[kLevels - 1] + 1e-3f;
+      if (target <= 0.99f) {
+        auto mass_above = [&](float t, int* cnt) {
+          float m = 0.f;
+          int c = 0;
 #pragma unroll
-        for (int t = kLevels - 1; t >= 0; --t)
-          if (c < a.tau[t]) l = t;
-        lev[j] = (int8_t)l;
-        c += __uint_as_float((unsigned)(v[r] >> 32));
+          for (int r = 0; r < K; ++r) {
+            const bool in = lane * K + r < nvis && pj[r] >= t;
+            m += in ? pj[r] : 0.f;
+            c += in;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            m += __shfl_xor_sync(0xffffffffu, m, o);
+            c += __shfl_xor_sync(0xffffffffu, c, o);
+          }
+          *cnt = c;
+          return m;
+        };
+        float pmax = 0.f;
+#pragma unroll
+        for (int r = 0; r < K; ++r) pmax = fmaxf(pmax, pj[r]);
+        pmax = warp_max(pmax);
+        int m_hi;
+        float lo = 0.f, hi = pmax, t;
+        int m;
+        if (mass_above(hi, &m_hi) >= target) {
+          t = hi;
+          m = m_hi;
+        } else {
+          int m_lo = nvis;                 // the whole row: mass 1 >= target
+          for (int it = 0; it < 40 && m_lo > kCand; ++it) {
+            const float mid = 0.5f * (lo + hi);
+            if (!(mid > lo && mid < hi)) break;
+            int c;
+            if (mass_above(mid, &c) >= target) {
+              lo = mid;
+              m_lo = c;
+            } else {
+              hi = mid;
+            }
+          }
+          t = lo;
+          m = m_lo;
+        }
+        if (m <= kCand) {
+          int mine = 0;
+#pragma unroll
+          for (int r = 0; r < K; ++r) mine += lane * K + r < nvis && pj[r] >= t;
+          int tot;
+          int pos = warp_excl_scan(mine, &tot);
+#pragma unroll
+          for (int r = 0; r < K; ++r) {
+            const int i = lane * K + r;
+            if (i < nvis && pj[r] >= t)
+              key[pos++] = ((unsigned long long)__float_as_uint(pj[r]) << 32) | (0xffffffffu - (unsigned)i);
+          }
+          __syncwarp();
+          // the running mass of a candidate is the mass of the candidates
+          // ranked before it: those with a larger key (P, then lower index)
+          unsigned long long mk[kCandPerLane];
+          float c[kCandPerLane];
+#pragma unroll
+          for (int r = 0; r < kCandPerLane; ++r) {
+            const int i = lane + 32 * r;
+            mk[r] = i < m ? key[i] : ~0ull;
+            c[r] = 0.f;
+          }
+          for (int jj = 0; jj < m; ++jj) {
+            const unsigned long long kj = key[jj];          // same address in every lane
+            const float pj_ = __uint_as_float((unsigned)(kj >> 32));
+#pragma unroll
+            for (int r = 0; r < kCandPerLane; ++r) c[r] += kj > mk[r] ? pj_ : 0.f;
+          }
+#pragma unroll
+          for (int r = 0; r < kCandPerLane; ++r) {
+            if (lane + 32 * r < m) {
+              const int j = (int)(0xffffffffu - (unsigned)(mk[r] & 0xffffffffu));
+              int l = -1;
+#pragma unroll
+              for (int t = kLevels - 1; t >= 0; --t)
+                if (c[r] < a.tau[t]) l = t;
+              lev[j] = (int8_t)l;
+            }
+          }
+          done = true;
+        }
       }
+    }
+    if (!done) {
+      // the whole row sorted in registers: lane L holds ranks L*K .. L*K + K - 1
+      unsigned long long v[K];
+#pragma unroll
+      for (int r = 0; r < K; ++r) {
+        const int i = lane * K + r;
+        v[r] = i < nvis ? ((unsigned long long)__float_as_uint(pj[r]) << 32) | (0xffffffffu - (unsigned)i)
+                        : 0ull;
+      }
+      warp_bitonic_desc<K>(v);
+      levels_from_sorted<K>(v, nvis, a.tau, lev);
     }
   } else {
     for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
@@ -336,8 +492,8 @@ __global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
   if (row >= nrows) return;
   const int lev_stride = (a.Nk + 15) & ~15;
   int8_t* lev = reinterpret_cast<int8_t*>(smem) + (size_t)warp * lev_stride;
-  for (int j = lane; j < a.Nk; j += 32) {
-    const int8_t v = map[(long long)row * a.Nk + j];
+  for (int j = lane; j < lev_stride; j += 32) {
+    const int8_t v = j < a.Nk ? map[(long long)row * a.Nk + j] : (int8_t)-1;
     lev[j] = (v >= 0 && v < kLevels) ? v : (int8_t)-1;
   }
   __syncwarp();
@@ -370,7 +526,8 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
   const MaskArgs a = make_mask_args(p, L, scale);
   const int n2 = next_pow2(L.Nk < 32 ? 32 : L.Nk);
   const bool in_regs = n2 <= 1024;          // register sort; larger rows sort in shared memory
-  const size_t per_row = (in_regs ? 0 : (size_t)n2 * 8) + ((L.Nk + 15) & ~15);
+  const int K = in_regs ? n2 / 32 : 0;
+  const size_t per_row = assign_key_bytes(K, n2) + ((L.Nk + 15) & ~15);
   int rows_per_cta = (int)((96 * 1024) / per_row);
   rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 2 ? 2 : rows_per_cta);
   const size_t smem = per_row * rows_per_cta;

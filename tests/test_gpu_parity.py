@@ -33,6 +33,18 @@ CASES = {
     # CUDA-core path, fp32, d = 128, 128-row query blocks
     "f32_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, dtype="f32",
                                  grid=(1, 18, 40), coarse=(1, 5, 10), seed=15, target="fixed"),
+    # 150 KV blocks per row (N = 9541, ragged): the assignment's candidate cut
+    # (a small tau_3, so only the top blocks are sorted)
+    "bf16_cand": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0, grid=(1, 47, 203),
+                                  coarse=(1, 12, 51), forced_prefix_tokens=0, seed=16,
+                                  target="alpha:0.15"),
+    # the same length, causal with grouped queries, through the candidate cut
+    "bf16_cand_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 47, 203),
+                                         coarse=(1, 12, 51), seed=17, target="alpha:0.3"),
+    # tau_3 = 1: every visible block is ranked, the full sort of the row
+    "bf16_full_sort": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0,
+                                       grid=(1, 47, 203), coarse=(1, 12, 51),
+                                       forced_prefix_tokens=0, seed=18, target="alpha:1.0"),
 }
 
 _cache = {}

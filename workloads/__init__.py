@@ -56,7 +56,7 @@ class Workload:
     causal: bool
     forced_prefix_tokens: int       # KV blocks holding any of these tokens get level 0
     seed: int
-    target: str                     # how tau is chosen: "fixed", "skip:0.91", "keep:0.35"
+    target: str                     # how tau is chosen: "fixed", "alpha:0.15", "skip:0.91", "keep:0.35"
     pool: Tuple[int, int, int, int] = (1, 2, 4, 8)
 
     @property
@@ -107,10 +107,14 @@ BY_NAME = {w.name: w for w in WORKLOADS}
 def thresholds(w: Workload) -> Tuple[float, float, float, float]:
     """The cumulative-mass thresholds tau_0..tau_3 of a workload.
 
-    The tiny case fixes them; the others read the alpha frozen in
-    ``thresholds.json`` (written by ``oracle/tune_thresholds.py``)."""
+    The tiny case fixes them; "alpha:X" scales the shape to tau_3 = X; the
+    others read the alpha frozen in ``thresholds.json`` (written by
+    ``oracle/tune_thresholds.py``)."""
     if w.target == "fixed":
         return TAU_SHAPE
+    if w.target.startswith("alpha:"):
+        alpha = float(w.target.split(":", 1)[1])
+        return tuple(float(alpha * t / TAU_SHAPE[-1]) for t in TAU_SHAPE)
     with open(THRESHOLDS_FILE) as f:
         alpha = json.load(f)[w.name]["alpha"]
     return tuple(float(alpha * t / TAU_SHAPE[-1]) for t in TAU_SHAPE)
