@@ -12,22 +12,27 @@
 // Each pooled key's logit gets + log2(c) (c = tokens it averages) so that it
 // carries their softmax mass.
 //
-// Persistent CTAs (one per SM) walk the query blocks; per query block, 10 warps:
+// Persistent CTAs (one per SM) walk the query blocks; 12 warps:
 //   warp 0     TMA producer for Q and K: Q once per query block; per tile, one
 //              2-D box per sub-block and 64-column half (the box height is the
 //              level's sub-block height), plus the tile's key bias table.
-//   warp 10    TMA producer for V, the same boxes into the V ring.
-//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer:
-//              S[t%2] = Q K_t^T (SS form), then O += P_t V_t with P read from
-//              TMEM (TS form); commits signal the softmax and free stages.
-//   warps 2-9  softmax, two warpgroups: each row is shared by one thread of
-//              each group (TMEM lane = row), which take 64 keys of the tile
-//              each; online softmax in log2 units with the partial row maxima
-//              exchanged per tile, P written back to TMEM as bf16, lazy O
-//              rescale (only when the running max grows by more than 2^8),
-//              epilogue O / lse split by column halves.
-// TMEM columns: S0 [0,128) S1 [128,256) (P(t) over S(t)), O [256,256+d),
-// Q [384,384+d/2): QK^T reads Q from TMEM, so shared memory only feeds K and V.
+//   warp 2     TMA producer for V, the same boxes into the V ring.
+//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer.
+//   warps 4-7, 8-11   softmax, one warpgroup per stream.
+// A query block's tiles alternate between two streams (even tiles, odd
+// tiles), each with its own S buffer and O accumulator in TMEM and its own
+// online softmax state, merged once at the end of the block (the two partial
+// softmaxes over disjoint key sets combine exactly).  The warpgroups never
+// wait for each other inside a block, so one computes exponentials while the
+// other waits for or loads its scores, and the tensor pipe always has the
+// other stream's QK^T or PV to run.  Per stream s and tile t (t = s mod 2):
+//   S_s = Q K_t^T (SS form; Q and K in shared memory),
+//   softmax(t): P_t = exp2(S_s * scale + bias - m_s), written over S_s (bf16),
+//   O_s += P_t V_t (TS form, P from TMEM), then QK^T of tile t + 2 into S_s
+//   (the in-order tensor pipe finishes PV(t) before it overwrites P_t).
+// Each row's logits get + log2(c) of the pooled key's token count; the
+// running maximum is rescaled lazily (only when it grows by more than 2^8).
+// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+d) O_1 [256+d,256+2d).
 // Every mbarrier wait is bounded: on expiry the kernel records a timeout in
 // the workspace error word and winds down without trapping.
 #include "psa_internal.cuh"
@@ -45,9 +50,10 @@ using namespace ptx;
 
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per packed tile
-constexpr int kSoftGroups = 2;    // softmax warpgroups sharing each tile (64 keys each)
-constexpr int kVWarp = 2 + 4 * kSoftGroups;        // the V producer, after the softmax warps
-constexpr int kThreads = 96 + 128 * kSoftGroups;   // K producer, MMA, softmax, V producer
+constexpr int kStreams = 2;              // softmax warpgroups, one per stream of tiles
+constexpr int kVWarp = 2;                // the V producer
+constexpr int kSoftWarp0 = 4;            // first softmax warp (warpgroup aligned)
+constexpr int kThreads = 128 + 128 * kStreams;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
@@ -68,8 +74,8 @@ struct Cfg {
   static constexpr int OFF_META = OFF_V + VSTAGES * KV_BYTES;   // per table: bias[128], kpos[128]
   static constexpr int META_BYTES = 128 + 1024;                // chunk biases, flag, per-key tables
   static constexpr int OFF_BAR = OFF_META + MSTAGES * META_BYTES;
-  static constexpr int OFF_XCH = OFF_BAR + 512;                 // softmax exchange [2][groups][128]
-  static constexpr int OFF_LIST = OFF_XCH + 2 * kSoftGroups * 512;   // the query block's work list
+  static constexpr int OFF_XCH = OFF_BAR + 512;                 // stream merge [2][streams][128][2]
+  static constexpr int OFF_LIST = OFF_XCH + 2 * kStreams * 128 * 8;  // the query block's work list
   static constexpr int SMEM = OFF_LIST + 2 * kListCache * 4 + 1024;   // two list copies + slack
 };
 
@@ -140,9 +146,7 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 }
 
 // How many of every 8 exponential pairs of a softmax tile take the FMA-pipe
-// polynomial above.  With one 128-row query tile per CTA the tensor-core
-// chain, not the transcendental unit, limits a tile (3 of 8 measured 2%
-// slower than 0 on the 1.3B video shape), so all go to the MUFU.
+// polynomial above, the rest the transcendental unit (MUFU).
 constexpr int kPolyPairs = 0;
 
 // ------------------------------------------------------------ work list
@@ -216,8 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   constexpr int B_KFULL = 2, B_KEMPTY = B_KFULL + KS;
   constexpr int B_VFULL = B_KEMPTY + KS, B_VEMPTY = B_VFULL + VS;
   constexpr int B_MFULL = B_VEMPTY + VS, B_MEMPTY = B_MFULL + MS;
-  constexpr int B_SFULL = B_MEMPTY + MS, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
-  constexpr int B_FINAL = B_ODONE + 2, NBARS = B_FINAL + 1;
+  constexpr int B_SFULL = B_MEMPTY + MS, B_PFULL = B_SFULL + kStreams;
+  constexpr int B_OFULL = B_PFULL + kStreams, B_OFREE = B_OFULL + 1;
+  constexpr int B_FINAL = B_OFREE + 1, NBARS = B_FINAL + 1;
   static_assert(NBARS * 8 + 16 <= 512, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -228,15 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
-    mbar_init(bar(B_QEMPTY), 128 * kSoftGroups);   // Q copied to TMEM (smem Q free)
+    mbar_init(bar(B_QEMPTY), 1);                     // the block's last QK^T completed
     for (int s = 0; s < KS; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
     for (int s = 0; s < VS; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
-    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 4 * kSoftGroups); }
-    for (int i = 0; i < 2; ++i) {
+    for (int s = 0; s < MS; ++s) { mbar_init(bar(B_MFULL + s), 32); mbar_init(bar(B_MEMPTY + s), 4); }
+    for (int i = 0; i < kStreams; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PFULL + i), 128 * kSoftGroups);
-      mbar_init(bar(B_ODONE + i), 1);
+      mbar_init(bar(B_PFULL + i), 128);
     }
+    mbar_init(bar(B_OFULL), 1);                      // the block's last PV completed
+    mbar_init(bar(B_OFREE), 128 * kStreams);         // both accumulators read out
     mbar_init(bar(B_FINAL), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -260,9 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S0 [0,128) S1 [128,256) (P(t) is written over S(t), as bf16
-  // pairs, once both softmax groups have read it), O [256, 256+D), Q [384, 384+D/2)
-  const uint32_t T_S = tmem, T_O = tmem + 256, T_Q = tmem + 384;
+  // TMEM columns: S_s [128 s, 128 s + 128) (P_t written over it as bf16 pairs),
+  // O_s [256 + D s, 256 + D s + D)
+  const uint32_t T_S = tmem, T_O = tmem + 256;
 
   if (warp == 0) {
     // ---------------------------------------------------- K / Q producer
@@ -401,59 +407,68 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_bf16(kBM, kBN, false);
       constexpr uint32_t ID_PV = idesc_bf16(kBM, D, true);
+      const uint64_t qdesc0 = sdesc(sbase + C::OFF_Q, 16, 1024);
       const uint64_t kdesc0 = sdesc(sbase + C::OFF_K, 16, 1024);
       const uint64_t vdesc0 = sdesc(sbase + C::OFF_V, C::HALF, 1024);
       bool ok = true;
-      auto issue_pv = [&](int u, bool first) -> bool {
-        const int s = u % VS, bb = u & 1;
-        if (!wait_bar(bar(B_PFULL + bb), (u >> 1) & 1, abort_flag, p.err)) return false;
-        if (!wait_bar(bar(B_VFULL + s), (u / VS) & 1, abort_flag, p.err)) return false;
-        tc_fence_after();
-        const uint64_t vd = vdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
-        const uint32_t dP = T_S + bb * 128;          // P(u) written over S(u)
-#pragma unroll
-        for (int k = 0; k < kBN / 16; ++k)
-          mma_ts(T_O, dP + k * 8, vd + (uint64_t)(k * (2048 >> 4)), ID_PV,
-                 (first && k == 0) ? 0u : 1u);
-        mma_commit(bar(B_ODONE + bb));
-        mma_commit(bar(B_VEMPTY + s));
-        return true;
-      };
-      // QK^T of tile u into S[u % 2].  That buffer was last read by the
-      // softmax of tile u - 2, which finished before P(u - 2) was ready, and
-      // PV(u - 2) (issued before this call) waited for P(u - 2).
-      auto issue_qk = [&](int u) -> bool {
-        const int s = u % KS, bb = u & 1;
+      int np[kStreams] = {0, 0};             // PVs issued per stream
+      // S_s = Q K^T of the tile with global index u (K stage u % KS)
+      auto issue_qk = [&](int u, int st) -> bool {
+        const int s = u % KS;
         if (!wait_bar(bar(B_KFULL + s), (u / KS) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
         // descriptors advance by adding the byte offset / 16 to the start-address field
         const uint64_t kd = kdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
-        const uint32_t dS = T_S + bb * 128;
+        const uint32_t dS = T_S + st * 128;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          constexpr uint32_t kHalfStep = C::HALF >> 4;
+          constexpr uint32_t kHalfStep = C::HALF >> 4;   // same layout for Q and K halves
           const uint64_t off = (uint64_t)((k >> 2) * kHalfStep + (k & 3) * 2);
-          mma_ts(dS, T_Q + k * 8, kd + off, ID_QK, k > 0 ? 1u : 0u);   // A = Q in TMEM
+          mma_ss(dS, qdesc0 + off, kd + off, ID_QK, k > 0 ? 1u : 0u);
         }
-        mma_commit(bar(B_SFULL + bb));
+        mma_commit(bar(B_SFULL + st));
         mma_commit(bar(B_KEMPTY + s));
         return true;
       };
-      // Order per query block: QK(0), then for each tile t >= 1: QK(t), PV(t - 1);
-      // finally PV(T - 1).  QK^T of the next tile runs while the softmax of the
-      // current one works.
+      // O_s += P V of the tile with global index u; P was written over S_s
+      auto issue_pv = [&](int u, int st, bool first) -> bool {
+        const int s = u % VS;
+        if (!wait_bar(bar(B_PFULL + st), np[st] & 1, abort_flag, p.err)) return false;
+        ++np[st];
+        if (!wait_bar(bar(B_VFULL + s), (u / VS) & 1, abort_flag, p.err)) return false;
+        tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)((s * C::KV_BYTES) >> 4);
+        const uint32_t dP = T_S + st * 128;
+        const uint32_t dO = T_O + st * D;
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          mma_ts(dO, dP + k * 8, vd + (uint64_t)(k * (2048 >> 4)), ID_PV,
+                 (first && k == 0) ? 0u : 1u);
+        mma_commit(bar(B_VEMPTY + s));
+        return true;
+      };
+      // Per query block: QK(0), QK(1); then for each tile t: PV(t), QK(t + 2).
       int g = 0, iq = 0;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
-        if (!wait_bar(bar(B_QEMPTY), iq & 1, abort_flag, p.err)) { ok = false; break; }   // Q in TMEM
+        if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
+        for (int t = 0; ok && t < 2 && t < T; ++t) {
+          ok = issue_qk(g + t, t);
+          if (ok && t == T - 1) mma_commit(bar(B_QEMPTY));   // the block's last QK^T
+        }
+        // both accumulators of the previous block have been read out
+        if (ok && iq > 0 && !wait_bar(bar(B_OFREE), (iq - 1) & 1, abort_flag, p.err)) ok = false;
         ++iq;
         for (int t = 0; ok && t < T; ++t) {
-          ok = issue_qk(g + t);
-          if (ok && t >= 1) ok = issue_pv(g + t - 1, t == 1);
+          ok = issue_pv(g + t, t & 1, t < 2);
+          if (ok && t + 2 < T) {
+            ok = issue_qk(g + t + 2, t & 1);
+            if (ok && t + 2 == T - 1) mma_commit(bar(B_QEMPTY));
+          }
         }
-        if (ok) ok = issue_pv(g + T - 1, T == 1);
         if (!ok) break;
+        mma_commit(bar(B_OFULL));
         g += T;
       }
       // drain: every MMA issued so far completes before TMEM is released
@@ -462,216 +477,210 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       while (!mbar_try_wait(bar(B_FINAL), 0) && global_ns() - t0 < kTimeoutNs) {
       }
     }
-  } else {
+  } else if (warp >= kSoftWarp0) {
     // --------------------------------------------------------------- softmax
-    // kSoftGroups warpgroups share every row: group hg takes keys
-    // [KW*hg, KW*hg + KW) of each tile and O columns [hg*HD, (hg+1)*HD).  The
-    // warps that own the same 32 rows (same TMEM lane quadrant) exchange
-    // their partial row maxima every tile through shared memory and a named
-    // barrier, so all keep the same running max; partial row sums are added
-    // at the end.  Every warp takes the same number of barriers on every path
-    // (also after a timed-out wait), so the barrier cannot hang.
-    constexpr int NG = kSoftGroups;
-    constexpr int KW = kBN / NG;        // keys per group and tile
-    constexpr int HD = D / NG;          // O columns per group
-    constexpr int OC = HD < 32 ? HD : 32;
-    const int hg = (warp - 2) >> 2;
+    // Warpgroup st owns stream st: tiles t = st, st + 2, ... of every query
+    // block.  Thread = query row r of the block (TMEM lane r).  The row's
+    // scores of a tile are read from S_st twice: pass 1 (all 128 at once)
+    // takes the tile maximum, pass 2 the exponentials, 64 keys at a time.  At the end of the block
+    // the two streams' (max, sum) are exchanged through shared memory and a
+    // named barrier (every warp takes it once per block, on every path), and
+    // each warpgroup writes half of the merged O columns.
+    const int st = (warp - kSoftWarp0) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][NG][128]
-    int nx = 0;                                                 // exchanges so far
-    // writes v, returns the NG values of this row (group order)
-    auto exchange = [&](float v, float (&all)[NG]) {
-      float* buf = xch + (nx & 1) * (NG * 128);
-      buf[hg * 128 + r] = v;
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "r"(32 * NG) : "memory");
-      ++nx;
-#pragma unroll
-      for (int i = 0; i < NG; ++i) all[i] = buf[i * 128 + r];
-    };
-    const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-    int g = 0, iqs = 0;
+    const uint32_t T_Ss = T_S + st * 128 + lane_off;
+    constexpr int HD = D / kStreams;         // merged O columns written by this warpgroup
+    constexpr int OC = HD < 32 ? HD : 32;
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][streams][128][2]
+    const float sc = p.scale_log2;
+    const uint64_t sc2 = f2pack(sc, sc);
+    int g = 0, ns = 0, nb = 0;               // tiles before this block, stream tiles, blocks with work
     bool ok = true;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int qpos = qa * kBM + r;
       float m = -INFINITY, lsum = 0.f;
-      if (T > 0) {
-        // Q of this query block into TMEM (the A operand of QK^T): row r,
-        // packed bf16 pairs [hg*D/4, (hg+1)*D/4) of the row, read out of the
-        // 128-byte-swizzled TMA tile.  The previous block's QK^T are complete
-        // (its last PV, which followed them, was waited for in the epilogue).
-        ok = ok && warp_wait(bar(B_QFULL), iqs & 1, abort_flag, p.err);
-        if (ok) {
-          constexpr int QW = D / 2 / NG;               // packed columns per group
-          uint32_t qv[QW];
-#pragma unroll
-          for (int c = 0; c < QW; c += 4) {
-            const int e = 2 * (hg * QW + c);             // first element of this 16-byte chunk
-            const int h = e >> 6, ch = (e & 63) >> 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                smem + C::OFF_Q + h * (kBM * 128) + r * 128 + ((ch ^ (r & 7)) << 4));
-            qv[c] = v.x; qv[c + 1] = v.y; qv[c + 2] = v.z; qv[c + 3] = v.w;
-          }
-          tmem_stn<QW>(T_Q + lane_off + hg * QW, qv);
-          tmem_st_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(bar(B_QEMPTY));
-        ++iqs;
-      }
-      for (int t = 0; t < T; ++t) {
-        const int gt = g + t, bb = gt & 1, ms = gt % MS;
-        ok = ok && warp_wait(bar(B_SFULL + bb), (gt >> 1) & 1, abort_flag, p.err) &&
+      for (int t = st; t < T; t += 2, ++ns) {
+        const int gt = g + t, ms = gt % MS;
+        ok = ok && warp_wait(bar(B_SFULL + st), ns & 1, abort_flag, p.err) &&
              warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err);
-        float x[KW];
-        float mt = -INFINITY;
-        if (ok) {
-          tc_fence_after();
-          const unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
-          const bool slow = *reinterpret_cast<const int*>(mt_base + 64) != 0;
-          const float* cb = reinterpret_cast<const float*>(mt_base) + (KW / 8) * hg;
-          const float* mbias = reinterpret_cast<const float*>(mt_base + 128) + KW * hg;
-          const int* mpos = reinterpret_cast<const int*>(mt_base + 128 + 512) + KW * hg;
-          tmem_ldn<KW>(T_S + bb * 128 + lane_off + KW * hg, reinterpret_cast<uint32_t*>(x));
-          float cbv[KW / 8];
-#pragma unroll
-          for (int i = 0; i < KW / 8; ++i) cbv[i] = cb[i];
+        if (!ok) continue;
+        tc_fence_after();
+        const unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
+        const bool slow = *reinterpret_cast<const int*>(mt_base + 64) != 0;
+        const float* cb = reinterpret_cast<const float*>(mt_base);            // [16] chunk biases
+        const float* mbias = reinterpret_cast<const float*>(mt_base + 128);   // [128]
+        const int* mpos = reinterpret_cast<const int*>(mt_base + 128 + 512);  // [128]
+        // scaled, biased (and causally masked) logits of keys [h*64, h*64+64)
+        auto logits = [&](float (&x)[64], int h) {
+          tmem_ldn<64>(T_Ss + 64 * h, reinterpret_cast<uint32_t*>(x));
           tmem_ld_wait();
-          reg_fence<KW>(reinterpret_cast<uint32_t*>(x));
-          float mx0 = -INFINITY, mx1 = -INFINITY;
+          reg_fence<64>(reinterpret_cast<uint32_t*>(x));
           if (!slow) {
 #pragma unroll
-            for (int c = 0; c < KW; c += 4) {
-              const float b = cbv[c >> 3];
-              const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b, b));
-              const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b, b));
-              f2unpack(v01, x[c], x[c + 1]);
-              f2unpack(v23, x[c + 2], x[c + 3]);
-              mx0 = fmax3(mx0, x[c], x[c + 1]);
-              mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+            for (int c = 0; c < 64; c += 2) {
+              const float b = cb[8 * h + (c >> 3)];
+              f2unpack(ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b, b)), x[c], x[c + 1]);
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < KW; c += 4) {
-              const float4 b4 = *reinterpret_cast<const float4*>(mbias + c);
-              const uint64_t v01 = ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b4.x, b4.y));
-              const uint64_t v23 = ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b4.z, b4.w));
-              f2unpack(v01, x[c], x[c + 1]);
-              f2unpack(v23, x[c + 2], x[c + 3]);
+            for (int c = 0; c < 64; c += 4) {
+              const float4 b4 = *reinterpret_cast<const float4*>(mbias + 64 * h + c);
+              f2unpack(ffma2(f2pack(x[c], x[c + 1]), sc2, f2pack(b4.x, b4.y)), x[c], x[c + 1]);
+              f2unpack(ffma2(f2pack(x[c + 2], x[c + 3]), sc2, f2pack(b4.z, b4.w)), x[c + 2], x[c + 3]);
               if (p.causal) {
-                const int4 k4 = *reinterpret_cast<const int4*>(mpos + c);
+                const int4 k4 = *reinterpret_cast<const int4*>(mpos + 64 * h + c);
                 if (qpos < k4.x) x[c] = -INFINITY;
                 if (qpos < k4.y) x[c + 1] = -INFINITY;
                 if (qpos < k4.z) x[c + 2] = -INFINITY;
                 if (qpos < k4.w) x[c + 3] = -INFINITY;
               }
+            }
+          }
+        };
+        // pass 1: the tile's row maximum.  In the common case every key of an
+        // 8-key chunk has the same bias, so the chunk's largest dot product
+        // gives its largest logit.
+        float mt = -INFINITY;
+        if (!slow) {
+          uint32_t v[128];
+          tmem_ldn<64>(T_Ss, v);
+          tmem_ldn<64>(T_Ss + 64, v + 64);
+          tmem_ld_wait();
+          reg_fence<128>(v);
+          float mc[16];
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            const float mx = fmax3(fmax3(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2])),
+                                   fmax3(__uint_as_float(v[c + 3]), __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5])),
+                                   fmaxf(__uint_as_float(v[c + 6]), __uint_as_float(v[c + 7])));
+            mc[c >> 3] = fmaf(mx, sc, cb[c >> 3]);   // -inf bias: the chunk holds no keys
+          }
+          mt = fmax3(fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmax3(mc[6], mc[7], mc[8])),
+                     fmax3(mc[9], mc[10], mc[11]), fmax3(mc[12], mc[13], fmaxf(mc[14], mc[15])));
+        } else {
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            float x[64];
+            logits(x, h);
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
               mx0 = fmax3(mx0, x[c], x[c + 1]);
               mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
             }
+            mt = fmaxf(mt, fmaxf(mx0, mx1));
           }
-          mt = fmaxf(mx0, mx1);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
         }
-        float parts[NG];
-        exchange(mt, parts);
-        if (!ok) continue;
-        mt = parts[0];
-#pragma unroll
-        for (int i = 1; i < NG; ++i) mt = fmaxf(mt, parts[i]);
         const float m_new = fmaxf(m, mt);
         const bool need = m_new > m + kRescaleLog2;     // false while both are -inf
         if (__any_sync(0xffffffffu, need)) {
           const float m_use = need ? m_new : m;
           const float factor = need ? ex2(m - m_use) : 1.f;   // 0 when m = -inf
-          if (t > 0) {
-            ok = warp_wait(bar(B_ODONE + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, abort_flag, p.err);
-            if (ok) {
-              tc_fence_after();
+          if (t >= 2) {
+            // O_st is quiescent: PV(t - 2) completed before S(t) was committed
 #pragma unroll
-              for (int c0 = 0; c0 < HD; c0 += OC) {
-                uint32_t o[OC];
-                tmem_ldn<OC>(T_O + lane_off + hg * HD + c0, o);
-                tmem_ld_wait();
-                reg_fence<OC>(o);
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(T_O + st * D + lane_off + c0, o);
+              tmem_ld_wait();
+              reg_fence<32>(o);
 #pragma unroll
-                for (int i = 0; i < OC; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                tmem_stn<OC>(T_O + lane_off + hg * HD + c0, o);
-              }
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+              tmem_st32(T_O + st * D + lane_off + c0, o);
             }
           }
           lsum *= factor;
           m = m_use;
         }
-        if (!ok) continue;
+        // pass 2: P = exp2(logit - m) as bf16 pairs, written over S_st
         const float m_base = m == -INFINITY ? 0.f : m;
         const uint64_t nm2 = f2pack(-m_base, -m_base);
         uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
-        uint32_t pk[KW / 2];
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float x[64];
+          logits(x, h);
+          uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < KW; c += 2) {
-          float p0, p1;
-          const uint64_t dd = fadd2(f2pack(x[c], x[c + 1]), nm2);
-          float d0, d1;
-          f2unpack(dd, d0, d1);
-          // kPolyPairs of every 8 pairs on the FMA pipes, interleaved with
-          // the rest on the transcendental unit
-          if (((c >> 1) & 7) < kPolyPairs) {
-            exp2_poly2(d0, d1, p0, p1);
-          } else {
-            p0 = ex2(d0);
-            p1 = ex2(d1);
+          for (int c = 0; c < 64; c += 2) {
+            float d0, d1, p0, p1;
+            f2unpack(fadd2(f2pack(x[c], x[c + 1]), nm2), d0, d1);
+            if (((c >> 1) & 7) < kPolyPairs) {
+              exp2_poly2(d0, d1, p0, p1);
+            } else {
+              p0 = ex2(d0);
+              p1 = ex2(d1);
+            }
+            if ((c >> 1) & 1) acc1 = fadd2(acc1, f2pack(p0, p1));
+            else acc0 = fadd2(acc0, f2pack(p0, p1));
+            __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+            pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
           }
-          if ((c >> 1) & 1) acc1 = fadd2(acc1, f2pack(p0, p1));
-          else acc0 = fadd2(acc0, f2pack(p0, p1));
-          __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
-          pk[c / 2] = *reinterpret_cast<uint32_t*>(&hh);
+          // P columns [32 h, 32 h + 32) overwrite logits this thread has read
+          tmem_stn<32>(T_Ss + 32 * h, pk);
         }
-        // P(gt - 2) in this buffer has been consumed: S(gt) was committed after
-        // PV(gt - 2) was issued, so its completion covers that PV.
-        tmem_stn<KW / 2>(T_S + bb * 128 + lane_off + (KW / 2) * hg, pk);   // P over S
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));   // bias table read
         float a0, a1, a2, a3;
         f2unpack(acc0, a0, a1);
         f2unpack(acc1, a2, a3);
         lsum += (a0 + a1) + (a2 + a3);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL + bb));
+        mbar_arrive(bar(B_PFULL + st));
       }
-      // epilogue of this query block: full row sum, then this group's O columns
-      float parts[NG];
-      exchange(lsum, parts);
-      float ltot = parts[0];
+      // ---- end of the query block: merge the two streams
+      float* xb = xch + (nb & 1) * (kStreams * 128 * 2);
+      xb[(st * 128 + r) * 2] = m;
+      xb[(st * 128 + r) * 2 + 1] = lsum;
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "r"(32 * kStreams) : "memory");
+      float ms_[kStreams], ls_[kStreams];
 #pragma unroll
-      for (int i = 1; i < NG; ++i) ltot += parts[i];
+      for (int i = 0; i < kStreams; ++i) {
+        ms_[i] = xb[(i * 128 + r) * 2];
+        ls_[i] = xb[(i * 128 + r) * 2 + 1];
+      }
+      const float M = fmaxf(ms_[0], ms_[1]);
+      const bool keys = M > -INFINITY;                  // the row kept at least one key
+      float f[kStreams], L = 0.f;
+#pragma unroll
+      for (int i = 0; i < kStreams; ++i) {
+        f[i] = ms_[i] > -INFINITY ? ex2(ms_[i] - M) : 0.f;
+        L += ls_[i] * f[i];
+      }
+      const float inv = keys ? 1.f / L : 0.f;
       const bool row_ok = qpos < p.N;
-      const bool keys = m > -INFINITY;                  // the row kept at least one key
-      const float inv = keys ? 1.f / ltot : 0.f;
-      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D + hg * HD;
-      const bool have_o = __all_sync(0xffffffffu, ok) && T > 0 &&
-                          warp_wait(bar(B_ODONE + ((g + T - 1) & 1)), ((g + T - 1) >> 1) & 1,
-                                    abort_flag, p.err);
+      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D + st * HD;
+      const bool have_o = T > 0 && __all_sync(0xffffffffu, ok) &&
+                          warp_wait(bar(B_OFULL), nb & 1, abort_flag, p.err);
       if (have_o) tc_fence_after();
 #pragma unroll
       for (int c0 = 0; c0 < HD; c0 += OC) {
-        uint32_t o[OC];
-        if (have_o) {
-          tmem_ldn<OC>(T_O + lane_off + hg * HD + c0, o);
-          tmem_ld_wait();
-          reg_fence<OC>(o);
-        } else {
+        float o[OC];
 #pragma unroll
-          for (int i = 0; i < OC; ++i) o[i] = 0u;
+        for (int i = 0; i < OC; ++i) o[i] = 0.f;
+        if (have_o) {
+#pragma unroll
+          for (int i = 0; i < kStreams; ++i) {
+            if (i < T) {                     // stream i holds tiles
+              uint32_t u[OC];
+              tmem_ldn<OC>(T_O + i * D + lane_off + st * HD + c0, u);
+              tmem_ld_wait();
+              reg_fence<OC>(u);
+#pragma unroll
+              for (int k = 0; k < OC; ++k) o[k] = fmaf(__uint_as_float(u[k]), f[i], o[k]);
+            }
+          }
         }
         if (row_ok) {
           uint32_t pk[OC / 2];
 #pragma unroll
           for (int i = 0; i < OC / 2; ++i) {
-            __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
-                                                      __uint_as_float(o[2 * i + 1]) * inv);
+            __nv_bfloat162 hh = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
             pk[i] = *reinterpret_cast<uint32_t*>(&hh);
           }
           uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
@@ -680,8 +689,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (row_ok && p.lse && hg == 0)
-        p.lse[(long long)bhq * p.N + qpos] = keys ? (m + log2f(ltot)) * kLn2 : -INFINITY;
+      if (row_ok && p.lse && st == 0)
+        p.lse[(long long)bhq * p.N + qpos] = keys ? (M + log2f(L)) * kLn2 : -INFINITY;
+      if (T > 0) {
+        // the accumulators may be overwritten by the next block's PVs
+        tc_fence_before();
+        mbar_arrive(bar(B_OFREE));
+        ++nb;
+      }
       g += T;
     }
   }
