@@ -50,14 +50,12 @@ def parse():
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# attention launch, from an ncu capture, keyed by the workload and a hash of
-# the attention kernel's sources.  A kernel that has changed since the
-# counters were taken has no entry, and the roofline's traffic is then null.
-# The Wan2.1-1.3B figure is a 6-head capture (278.1 MB) scaled by 2 to the
-# 12-head launch: every head reads its own Q, K and V levels once, so the
-# traffic grows in proportion to the heads.
+# attention launch, from an ncu capture of that launch, keyed by the workload,
+# its query heads and a hash of the attention kernel's sources.  A kernel that
+# has changed since the counters were taken has no entry, and the roofline's
+# traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "c6b363e67eeee4ae"): 2 * (236.379136e6 + 41.732096e6)}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "2ee739a4de2f4460"): 471.842304e6 + 92.477952e6}
 
 
 def attn_source_hash() -> str:
