@@ -127,7 +127,8 @@ def pyramid_bytes(w: W.Workload) -> float:
 
 def cpu_sample(w: W.Workload, n_heads: int):
     """Time the oracle (as it stands) on `n_heads` whole heads of the workload.
-    Returns (dense-equivalent TFLOP/s, seconds, cores, sample description)."""
+    Returns (dense-equivalent TFLOP/s, seconds, cores, sample description,
+    the oracle's per-head results)."""
     import oracle as O
     cores = len(os.sched_getaffinity(0))
     grp = w.Hq // w.Hkv
@@ -135,14 +136,41 @@ def cpu_sample(w: W.Workload, n_heads: int):
     inp = W.make_inputs(w, heads_q=heads, heads_kv=sorted({h // grp for h in heads}))
     tau = W.thresholds(w)
     t0 = time.perf_counter()
+    results = []
     for h in heads:
-        O.psa_head(inp.as_f64("q", 0, h), inp.as_f64("k", 0, h // grp), inp.as_f64("v", 0, h // grp),
-                   w.q_blk, w.kv_blk, tau, w.causal, w.forced_prefix_tokens)
+        results.append(O.psa_head(inp.as_f64("q", 0, h), inp.as_f64("k", 0, h // grp),
+                                  inp.as_f64("v", 0, h // grp), w.q_blk, w.kv_blk, tau, w.causal,
+                                  w.forced_prefix_tokens))
     dt = time.perf_counter() - t0
     dense = w.dense_flops() / (w.B * w.Hq) * n_heads
     return (dense / dt / 1e12, dt, cores,
             f"{n_heads} of {w.B * w.Hq} heads of {w.name}, whole forward (pyramid, mask, attention), "
-            f"NumPy float64, BLAS threads = {cores}")
+            f"NumPy float64, BLAS threads = {cores}", results)
+
+
+def sampled_parity(w: W.Workload, results, level_map, out) -> dict:
+    """GPU against the oracle on the sampled heads (batch 0): level-map entries
+    that differ, and the output error over the query blocks whose map rows
+    agree (so both sides attend to the same keys).  The tests hold the full
+    criterion (near-threshold and near-tie exemptions); this is a summary."""
+    mism, n_map, err_max, num, den = 0, 0, 0.0, 0.0, 0.0
+    for h, r in enumerate(results):
+        gm = level_map[0, h].cpu().numpy()
+        om = r.mask.level_map
+        mism += int((gm != om).sum())
+        n_map += om.size
+        same = np.all(gm == om, axis=1)
+        rows = np.concatenate([np.arange(a * w.q_blk, min((a + 1) * w.q_blk, w.N))
+                               for a in np.nonzero(same)[0]] or [np.zeros(0, dtype=np.int64)])
+        g = out[0, h].float().cpu().numpy().astype(np.float64)[rows]
+        ref = r.O[rows]
+        d = np.abs(g - ref)
+        err_max = max(err_max, float(d.max()) if d.size else 0.0)
+        num += float(d.sum())
+        den += float(np.abs(ref).sum())
+    return {"heads": len(results), "map_entries_differing": mism, "map_entries": n_map,
+            "max_abs": err_max, "mean_rel": num / den if den else 0.0,
+            "note": "output compared on query blocks whose GPU and oracle map rows agree"}
 
 
 def run_reference(args, rank, world):
@@ -153,7 +181,7 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         cpu_sample(w, 1)
     for _ in range(args.steps):
-        val, dt, cores, sample = cpu_sample(w, 1)
+        val, dt, cores, sample, _ = cpu_sample(w, 1)
         times.append(dt)
     tot = sum(times)
     dense_head = w.dense_flops() / (w.B * w.Hq)
@@ -323,11 +351,12 @@ def run_ours(args, rank, world, local_rank):
     mask_gbs = mask_bytes(w) / (mask_avg * 1e-3) / 1e9
     if rank != 0:
         return
-    cpu = None
+    cpu, parity = None, None
     if not args.no_cpu_baseline and world == 1:
-        val, dt, cores, sample = cpu_sample(w, args.cpu_sample_heads)
+        val, dt, cores, sample, results = cpu_sample(w, args.cpu_sample_heads)
         cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(dt, 2)}
+        parity = sampled_parity(w, results, lm, out)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -351,6 +380,7 @@ def run_ours(args, rank, world, local_rank):
                      "executed_flops_per_launch": executed,
                      "padding_fraction": 1.0 - (keys_per_row.sum() / max(padded_keys, 1.0))},
         "cpu_baseline": cpu,
+        "parity": parity,
         "e2e": {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * es),

@@ -163,6 +163,20 @@ psa_status_t psa_forward_noalloc(const psa_params_t* params, const void* Q, cons
 psa_status_t psa_check_device(const psa_params_t* params, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Failure-path self-test; the method has no counterpart.  Enqueues on
+ * `stream` one warp that waits, through the same bounded-wait code as the
+ * tensor-core kernels, on a barrier that nothing ever arrives at, and gives
+ * up after `limit_ns` nanoseconds (1 ns .. 1 s), recording a timeout in the
+ * workspace's device error word exactly as a kernel that timed out would.
+ * The next psa_check_device then returns PSA_ERR_DEVICE_TIMEOUT (and clears
+ * the word).  Nothing faults or traps.  params: any valid description whose
+ * workspace layout `workspace` holds; workspace: device, 256-byte aligned, at
+ * least psa_workspace_size(params) bytes (PSA_ERR_WORKSPACE_TOO_SMALL,
+ * PSA_ERR_MISALIGNED otherwise).  Returns PSA_ERR_INVALID_ARG for a null
+ * argument or a limit outside 1 ns .. 1 s, PSA_ERR_CUDA for a launch error. */
+psa_status_t psa_selftest_wait_timeout(const psa_params_t* params, void* workspace,
+                                       size_t workspace_bytes, uint64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 const char* psa_status_string(psa_status_t status);
 

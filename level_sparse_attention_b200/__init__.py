@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "psa_check_device": (ctypes.c_int, [P, vp, sz, vp]),
             "psa_forward_noalloc": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp]),
             "psa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "psa_selftest_wait_timeout": (ctypes.c_int, [P, vp, sz, ctypes.c_uint64, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -70,7 +71,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
             "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string",
-            "psa_forward_noalloc")
+            "psa_forward_noalloc", "psa_selftest_wait_timeout")
 
 
 def status_string(status: int) -> str:
@@ -156,6 +157,14 @@ def forward_noalloc(p: Params, Q, K, V, O, lse=None, level_map=None, stream=None
 def check_device(p: Params, ws: torch.Tensor, stream=None):
     _check(lib().psa_check_device(ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
            "psa_check_device")
+
+
+def selftest_wait_timeout(p: Params, ws: torch.Tensor, limit_ns: int, stream=None):
+    """Enqueue the failure-path self-test: a bounded wait that runs out after
+    ``limit_ns`` and records a timeout in the workspace's error word, which
+    the next check_device reports as PSA_ERR_DEVICE_TIMEOUT."""
+    _check(lib().psa_selftest_wait_timeout(ctypes.byref(p), _ptr(ws), ws.numel(), int(limit_ns),
+                                           _stream(stream)), "psa_selftest_wait_timeout")
 
 
 def map_shape(p: Params) -> Tuple[int, int, int, int]:

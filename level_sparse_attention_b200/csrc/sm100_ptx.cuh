@@ -41,21 +41,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on phase `parity` of `bar`.  Returns false when the CTA is
-// winding down (this or another role timed out).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* err) {
+// Bounded wait on phase `parity` of `bar`, giving up after `limit_ns`.
+// Returns false when the CTA is winding down (this or another role timed
+// out); a timeout sets the CTA's abort flag and the workspace error word.
+__device__ __forceinline__ bool wait_bar_ns(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            int* err, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > kTimeoutNs) {
+    if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(err, kErrTimeout);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int* err) {
+  return wait_bar_ns(bar, parity, abort_flag, err, kTimeoutNs);
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase.

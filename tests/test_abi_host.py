@@ -77,6 +77,21 @@ def test_argument_errors_before_any_launch():
     assert P.lib().psa_attention_fwd(ctypes.byref(p), A, A, A, B, need, None, A, mis, None) == 3
 
 
+def test_selftest_argument_errors_before_any_launch():
+    p = P.make_params(1, 2, 2, 1024, 64)
+    need = P.workspace_size(p)
+    st = lambda ws, n, limit: P.lib().psa_selftest_wait_timeout(ctypes.byref(p), ws, n, limit, None)
+    B = ctypes.c_void_p(0x20000)
+    assert st(B, need, 0) == 1                                      # limit out of range
+    assert st(B, need, 2_000_000_000) == 1
+    assert st(None, need, 1000) == 1                                # NULL workspace
+    assert st(ctypes.c_void_p(0x20010), need, 1000) == 3            # not 256-byte aligned
+    assert st(B, need - 1, 1000) == 4                               # too small
+    bad = P.make_params(1, 2, 2, 1024, 64)
+    bad.N = 0
+    assert P.lib().psa_selftest_wait_timeout(ctypes.byref(bad), B, need, 1000, None) == 1
+
+
 def test_status_strings():
     for s in range(7):
         assert P.status_string(s)
