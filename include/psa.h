@@ -50,23 +50,35 @@ typedef enum {
 
 typedef enum { PSA_F32 = 0, PSA_BF16 = 1 } psa_dtype_t;
 
+/* Level assignment rule (see psa_params_t.assign). */
+typedef enum { PSA_ASSIGN_THRESHOLD = 0, PSA_ASSIGN_QUANTILE = 1 } psa_assign_t;
+
 /* Problem description, shared by every entry point.
  *  B, Hq, Hkv, N, d  batch, query heads, KV heads (Hq % Hkv == 0; query head h
  *                    reads KV head h / (Hq / Hkv)), tokens, head dim (64 or 128).
  *  q_blk, kv_blk     query block (64 or 128) and KV block (64) sizes, in tokens.
  *  n_levels, pool    must be 4 and {1, 2, 4, 8}: level l pools 2^l tokens
  *                    ("Psa Pyramid Sparse Attention", Core Technique).
- *  tau               cumulative-mass thresholds, non-decreasing, in (0, 1]:
- *                    a KV block ranked r gets the smallest level l with
- *                    C_r < tau[l] (C_r = mass of the blocks ranked before it),
- *                    else it is pruned.
+ *  tau               non-decreasing, in (0, 1].  With assign = PSA_ASSIGN_THRESHOLD
+ *                    they are cumulative-mass thresholds: a KV block ranked r
+ *                    gets the smallest level l with C_r < tau[l] (C_r = mass of
+ *                    the blocks ranked before it), else it is pruned.  With
+ *                    assign = PSA_ASSIGN_QUANTILE they are cumulative fractions
+ *                    of the query block's visible KV blocks: the block ranked r
+ *                    (0-based) gets the smallest l with r < K_l, K_l =
+ *                    ceil(tau[l] * n_visible) computed exactly from the float
+ *                    value, else it is pruned.
  *  causal            1: key position <= query position (blocks after the query
  *                    block are pruned, blocks straddling its diagonal get level
  *                    0 and a token mask).
  *  forced_prefix_tokens  visible KV blocks holding any of the first this-many
  *                    tokens get level 0 (e.g. a text prefix).
  *  scale             softmax scale; 0 means 1/sqrt(d).
- *  dtype             element type of Q, K, V, O and of the pooled levels.    */
+ *  dtype             element type of Q, K, V, O and of the pooled levels.
+ *  assign            level assignment rule (psa_assign_t): threshold on the
+ *                    cumulative mass (the method's rule) or per-level quotas of
+ *                    blocks by rank (the quantile-based rule the method is
+ *                    compared with: top168.com article on PSA, ablations).   */
 typedef struct {
   int B, Hq, Hkv, N, d;
   int q_blk, kv_blk;
@@ -77,6 +89,7 @@ typedef struct {
   int forced_prefix_tokens;
   float scale;
   psa_dtype_t dtype;
+  psa_assign_t assign;
 } psa_params_t;
 
 /* Bytes of device workspace the calls below need for `params` (0 if params are

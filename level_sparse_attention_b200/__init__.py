@@ -36,7 +36,7 @@ class Params(ctypes.Structure):
                 ("kv_blk", ctypes.c_int), ("n_levels", ctypes.c_int),
                 ("pool", ctypes.c_int * 4), ("tau", ctypes.c_float * 4),
                 ("causal", ctypes.c_int), ("forced_prefix_tokens", ctypes.c_int),
-                ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("assign", ctypes.c_int)]
 
 
 _lib = None
@@ -81,10 +81,13 @@ def status_string(status: int) -> str:
         return _STATUS.get(status, "unknown")
 
 
+ASSIGN_THRESHOLD, ASSIGN_QUANTILE = 0, 1
+
+
 def make_params(B: int, Hq: int, Hkv: int, N: int, d: int, q_blk: int = 128, kv_blk: int = 64,
                 tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97), causal: bool = False,
                 forced_prefix_tokens: int = 0, scale: float = 0.0,
-                dtype: torch.dtype = torch.bfloat16) -> Params:
+                dtype: torch.dtype = torch.bfloat16, assign: int = ASSIGN_THRESHOLD) -> Params:
     p = Params()
     p.B, p.Hq, p.Hkv, p.N, p.d = B, Hq, Hkv, N, d
     p.q_blk, p.kv_blk, p.n_levels = q_blk, kv_blk, 4
@@ -93,6 +96,7 @@ def make_params(B: int, Hq: int, Hkv: int, N: int, d: int, q_blk: int = 128, kv_
         p.tau[i] = float(tau[i])
     p.causal, p.forced_prefix_tokens, p.scale = int(bool(causal)), forced_prefix_tokens, scale
     p.dtype = BF16 if dtype == torch.bfloat16 else F32
+    p.assign = int(assign)
     return p
 
 

@@ -249,11 +249,37 @@ __host__ __device__ inline size_t assign_key_bytes(int K, int n2) {
   return K == 0 ? (size_t)n2 * 8 : (K > kCandPerLane ? (size_t)kCand * 8 : 0);
 }
 
+// The level of a visible block from its place in the ranking.  Threshold
+// rule: the smallest l whose tau_l is above c, the mass of the blocks ranked
+// before it.  Quantile rule: the smallest l with rank < K_l, where K_l =
+// ceil(tau_l * n_visible) is computed exactly in double (a float times an
+// integer below 2^14 is exact there).
+struct LevelRule {
+  bool quantile;
+  float tau[kLevels];
+  int quota[kLevels];
+  __device__ LevelRule(const MaskArgs& a, int nvis) {
+    quantile = a.assign == PSA_ASSIGN_QUANTILE;
+#pragma unroll
+    for (int l = 0; l < kLevels; ++l) {
+      tau[l] = a.tau[l];
+      quota[l] = (int)ceil((double)a.tau[l] * (double)nvis);
+    }
+  }
+  __device__ __forceinline__ int8_t level(float c, int rank) const {
+    int l = -1;
+#pragma unroll
+    for (int t = kLevels - 1; t >= 0; --t)
+      if (quantile ? rank < quota[t] : c < tau[t]) l = t;
+    return (int8_t)l;
+  }
+};
+
 // Sorted keys (descending; lane L holds ranks L*K .. L*K + K - 1) -> levels of
-// the first n ranks: exclusive running mass c, level = first tau above c.
+// the first n ranks, with the exclusive running mass c of each.
 template <int K>
 __device__ __forceinline__ void levels_from_sorted(const unsigned long long (&v)[K], int n,
-                                                   const float* tau, int8_t* lev) {
+                                                   const LevelRule& rule, int8_t* lev) {
   const int lane = threadIdx.x & 31;
   float mine = 0.f;
 #pragma unroll
@@ -265,11 +291,7 @@ __device__ __forceinline__ void levels_from_sorted(const unsigned long long (&v)
   for (int r = 0; r < K; ++r) {
     if (lane * K + r < n) {
       const int j = (int)(0xffffffffu - (unsigned)(v[r] & 0xffffffffu));
-      int l = -1;
-#pragma unroll
-      for (int t = kLevels - 1; t >= 0; --t)
-        if (c < tau[t]) l = t;
-      lev[j] = (int8_t)l;
+      lev[j] = rule.level(c, lane * K + r);
       c += __uint_as_float((unsigned)(v[r] >> 32));
     }
   }
@@ -297,6 +319,7 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   const int q_hi = min(a.N, q_lo + a.q_blk) - 1;
   const int nvis = a.causal ? min(a.Nk, q_hi / a.kv_blk + 1) : a.Nk;
   const float* z = zlog + (long long)row * a.Nk;
+  const LevelRule rule(a, nvis);
 
   // softmax over the visible blocks
   float mx = -INFINITY;
@@ -312,8 +335,8 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   };
   for (int j = lane; j < lev_stride; j += 32) lev[j] = -1;
 
-  // rank by P descending (ties to the lower index), exclusive running mass,
-  // level = first tau the running mass is below
+  // rank by P descending (ties to the lower index); the level from the
+  // exclusive running mass (threshold rule) or the rank (quantile rule)
   if constexpr (K > 0) {
     // P of element i = lane*K + r in register r (0 past the visible blocks)
     float pj[K];
@@ -325,14 +348,16 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
     __syncwarp();                          // lev[] initialised by all lanes
     bool done = false;
     if constexpr (K > kCandPerLane) {
-      // Candidate cut: blocks with P >= t form a prefix of the ranking, and
-      // when their mass reaches tau_3 every block after them has a running
-      // mass >= tau_3, i.e. is pruned.  t is bisected until the candidates
-      // number at most kCand, with a margin of 1e-3 on the mass so that the
-      // rounding of this sum against the scan below cannot matter; then
-      // only the candidates are sorted.
+      // Candidate cut: blocks with P >= t form a prefix of the ranking.
+      // Threshold rule: when their mass reaches tau_3 every block after them
+      // has a running mass >= tau_3, i.e. is pruned (a margin of 1e-3 on the
+      // mass keeps the rounding of this sum against the running masses below
+      // from mattering).  Quantile rule: when they number at least K_3, every
+      // block after them has rank >= K_3.  t is bisected until the candidates
+      // number at most kCand; then only the candidates are ranked.
       const float target = a.tau[kLevels - 1] + 1e-3f;
-      if (target <= 0.99f) {
+      const int kq = rule.quota[kLevels - 1];
+      if (rule.quantile ? kq <= kCand : target <= 0.99f) {
         auto mass_above = [&](float t, int* cnt) {
           float m = 0.f;
           int c = 0;
@@ -354,19 +379,24 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
 #pragma unroll
         for (int r = 0; r < K; ++r) pmax = fmaxf(pmax, pj[r]);
         pmax = warp_max(pmax);
+        // do the blocks with P >= t reach past every kept rank?
+        auto enough = [&](float t, int* cnt) {
+          const float mass = mass_above(t, cnt);
+          return rule.quantile ? *cnt >= kq : mass >= target;
+        };
         int m_hi;
         float lo = 0.f, hi = pmax, t;
         int m;
-        if (mass_above(hi, &m_hi) >= target) {
+        if (enough(hi, &m_hi)) {
           t = hi;
           m = m_hi;
         } else {
-          int m_lo = nvis;                 // the whole row: mass 1 >= target
+          int m_lo = nvis;                 // the whole row: mass 1 >= target, nvis >= K_3
           for (int it = 0; it < 40 && m_lo > kCand; ++it) {
             const float mid = 0.5f * (lo + hi);
             if (!(mid > lo && mid < hi)) break;
             int c;
-            if (mass_above(mid, &c) >= target) {
+            if (enough(mid, &c)) {
               lo = mid;
               m_lo = c;
             } else {
@@ -389,31 +419,33 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
               key[pos++] = ((unsigned long long)__float_as_uint(pj[r]) << 32) | (0xffffffffu - (unsigned)i);
           }
           __syncwarp();
-          // the running mass of a candidate is the mass of the candidates
-          // ranked before it: those with a larger key (P, then lower index)
+          // a candidate's rank is the number of candidates with a larger key
+          // (P, then lower index), its running mass their total P
           unsigned long long mk[kCandPerLane];
           float c[kCandPerLane];
+          int rk[kCandPerLane];
 #pragma unroll
           for (int r = 0; r < kCandPerLane; ++r) {
             const int i = lane + 32 * r;
             mk[r] = i < m ? key[i] : ~0ull;
             c[r] = 0.f;
+            rk[r] = 0;
           }
           for (int jj = 0; jj < m; ++jj) {
             const unsigned long long kj = key[jj];          // same address in every lane
             const float pj_ = __uint_as_float((unsigned)(kj >> 32));
 #pragma unroll
-            for (int r = 0; r < kCandPerLane; ++r) c[r] += kj > mk[r] ? pj_ : 0.f;
+            for (int r = 0; r < kCandPerLane; ++r) {
+              const bool before = kj > mk[r];
+              c[r] += before ? pj_ : 0.f;
+              rk[r] += before;
+            }
           }
 #pragma unroll
           for (int r = 0; r < kCandPerLane; ++r) {
             if (lane + 32 * r < m) {
               const int j = (int)(0xffffffffu - (unsigned)(mk[r] & 0xffffffffu));
-              int l = -1;
-#pragma unroll
-              for (int t = kLevels - 1; t >= 0; --t)
-                if (c[r] < a.tau[t]) l = t;
-              lev[j] = (int8_t)l;
+              lev[j] = rule.level(c[r], rk[r]);
             }
           }
           done = true;
@@ -430,7 +462,7 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
                         : 0ull;
       }
       warp_bitonic_desc<K>(v);
-      levels_from_sorted<K>(v, nvis, a.tau, lev);
+      levels_from_sorted<K>(v, nvis, rule, lev);
     }
   } else {
     for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
@@ -458,11 +490,7 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
     for (int r = r0; r < r1; ++r) {
       const float pr = __uint_as_float((unsigned)(key[r] >> 32));
       const int j = (int)(0xffffffffu - (unsigned)(key[r] & 0xffffffffu));
-      int l = -1;
-#pragma unroll
-      for (int t = kLevels - 1; t >= 0; --t)
-        if (c < a.tau[t]) l = t;
-      lev[j] = (int8_t)l;
+      lev[j] = rule.level(c, r);
       c += pr;
     }
   }

@@ -24,6 +24,7 @@ psa_status_t validate(const psa_params_t* p) {
   }
   if (!(p->scale >= 0.f) || isinf(p->scale)) return PSA_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return PSA_ERR_INVALID_ARG;
+  if (p->assign != PSA_ASSIGN_THRESHOLD && p->assign != PSA_ASSIGN_QUANTILE) return PSA_ERR_INVALID_ARG;
   if (p->forced_prefix_tokens < 0) return PSA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return PSA_ERR_UNSUPPORTED;
   if (p->kv_blk != 64) return PSA_ERR_UNSUPPORTED;

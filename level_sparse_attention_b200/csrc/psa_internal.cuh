@@ -69,6 +69,7 @@ inline __host__ __device__ Layout make_layout(const psa_params_t& p) {
 struct MaskArgs {
   int B, Hq, Hkv, N, d, q_blk, kv_blk, Nq, Nk;
   int causal, forced_prefix_tokens;
+  int assign;                 // psa_assign_t
   float scale;
   float tau[kLevels];
 };
@@ -78,6 +79,7 @@ inline MaskArgs make_mask_args(const psa_params_t& p, const Layout& L, float sca
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.N = p.N; a.d = p.d;
   a.q_blk = p.q_blk; a.kv_blk = p.kv_blk; a.Nq = L.Nq; a.Nk = L.Nk;
   a.causal = p.causal; a.forced_prefix_tokens = p.forced_prefix_tokens;
+  a.assign = (int)p.assign;
   a.scale = scale;
   for (int l = 0; l < kLevels; ++l) a.tau[l] = p.tau[l];
   return a;

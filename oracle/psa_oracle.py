@@ -180,6 +180,23 @@ def level_of(c: np.ndarray, tau: Sequence[float]) -> np.ndarray:
     return out
 
 
+def quotas(n_visible: int, tau: Sequence[float]) -> np.ndarray:
+    """Quantile rule: K_l = ceil(tau_l * n_visible), the number of top-ranked
+    blocks at level <= l.  tau is taken at the single precision the C
+    interface carries it in, and the product is exact in float64 (a 24-bit
+    significand times an integer below 2^14)."""
+    t = np.asarray(tau, dtype=np.float32).astype(np.float64)
+    return np.ceil(t * float(n_visible)).astype(np.int64)
+
+
+def level_of_rank(rank: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """Quantile rule: level = the smallest l with rank < K_l, else pruned (-1)."""
+    out = np.full(rank.shape, PRUNED, dtype=np.int8)
+    for l in reversed(range(len(K))):
+        out[rank < K[l]] = l
+    return out
+
+
 def apply_overrides(row: np.ndarray, a: int, N: int, bq: int, bk: int, causal: bool,
                     forced_prefix_tokens: int) -> None:
     """In place: causal blocks after the query block are pruned and blocks
@@ -195,15 +212,22 @@ def apply_overrides(row: np.ndarray, a: int, N: int, bq: int, bk: int, causal: b
 
 
 def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
-                  causal: bool = False, forced_prefix_tokens: int = 0) -> MaskResult:
-    """Threshold-based multi-level mask ([news] ablations: threshold-based
-    assignment; [abs] lower levels to critical blocks, higher to less important).
+                  causal: bool = False, forced_prefix_tokens: int = 0,
+                  rule: str = "threshold") -> MaskResult:
+    """Multi-level mask ([news] ablations: threshold-based assignment, compared
+    there with a quantile-based one; [abs] lower levels to critical blocks,
+    higher to less important).
 
     For each query block a: P = softmax over visible j of z[a, j]; rank blocks by
-    P descending, ties to the lower j; C_r = mass of the blocks ranked before r;
-    level = the smallest l with C_r < tau_l, else pruned.  Then the overrides of
-    ``apply_overrides``.  Readings: the exclusive cumulative mass (so the top
-    block always gets level 0) and the override order are this build's."""
+    P descending, ties to the lower j; C_r = mass of the blocks ranked before r.
+    Threshold rule: level = the smallest l with C_r < tau_l, else pruned.
+    Quantile rule: level = the smallest l with r < K_l = ceil(tau_l * n_visible)
+    (``quotas``), else pruned.  Then the overrides of ``apply_overrides``.
+    Readings: the exclusive cumulative mass (so the top block always gets
+    level 0), the quotas as cumulative fractions of the visible blocks rounded
+    up, and the override order are this build's."""
+    if rule not in ("threshold", "quantile"):
+        raise ValueError(rule)
     Nq, Nk = z.shape
     level_map = np.full((Nq, Nk), PRUNED, dtype=np.int8)
     mass = np.zeros((Nq, Nk), dtype=np.float64)
@@ -214,7 +238,10 @@ def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
         order, p, c = rank_blocks(z[a], vis)
         mass[a, order], cum[a, order] = p, c
         rank[a, order] = np.arange(len(order))
-        level_map[a, order] = level_of(c, tau)
+        if rule == "threshold":
+            level_map[a, order] = level_of(c, tau)
+        else:
+            level_map[a, order] = level_of_rank(np.arange(len(order)), quotas(len(order), tau))
         apply_overrides(level_map[a], a, N, bq, bk, causal, forced_prefix_tokens)
     return MaskResult(level_map, mass, cum, rank)
 
@@ -282,7 +309,7 @@ class HeadResult:
 def psa_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, bq: int, bk: int,
              tau: Sequence[float], causal: bool = False, forced_prefix_tokens: int = 0,
              scale: Optional[float] = None, level_map: Optional[np.ndarray] = None,
-             pool: Sequence[int] = POOL) -> HeadResult:
+             pool: Sequence[int] = POOL, rule: str = "threshold") -> HeadResult:
     """The whole PSA forward for one (batch, query head): pyramid, query-block
     means, block logits, level assignment (unless ``level_map`` is given), then
     pyramid attention.  Q [N, d]; K, V [N, d] of the matching KV head."""
@@ -290,7 +317,7 @@ def psa_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, bq: int, bk: int,
     s = 1.0 / math.sqrt(d) if scale is None else scale
     pyr = build_pyramid(K, V, pool)
     z = block_logits(query_block_means(Q, bq), pyr, bk, s, pool)
-    mask = assign_levels(z, tau, N, bq, bk, causal, forced_prefix_tokens)
+    mask = assign_levels(z, tau, N, bq, bk, causal, forced_prefix_tokens, rule)
     lm = mask.level_map if level_map is None else level_map
     O, lse = pyramid_attention(Q, pyr, lm, bq, bk, s, causal, pool)
     return HeadResult(O, lse, mask, z)

@@ -7,6 +7,8 @@ log of sum over the block's level-3 keys of c_g * exp(s * qbar . k_g); softmax
 over visible blocks; rank by (-P, j); exclusive running mass; threshold cut;
 causal / forced overrides; per-row softmax over the kept keys with ln c_g."""
 import math
+import struct
+from fractions import Fraction
 
 
 def _mean(rows):
@@ -18,7 +20,7 @@ def _dot(a, b):
     return sum(x * y for x, y in zip(a, b))
 
 
-def psa_bruteforce(Q, K, V, bq, bk, tau, causal=False, forced=0, scale=None):
+def psa_bruteforce(Q, K, V, bq, bk, tau, causal=False, forced=0, scale=None, rule="threshold"):
     N, d = len(Q), len(Q[0])
     s = 1.0 / math.sqrt(d) if scale is None else scale
     pools = (1, 2, 4, 8)
@@ -53,10 +55,15 @@ def psa_bruteforce(Q, K, V, bq, bk, tau, causal=False, forced=0, scale=None):
         P = {j: w[j] / tw for j in vis}
         ranked = sorted(vis, key=lambda j: (-P[j], j))
         c = 0.0
-        for j in ranked:
+        # quantile rule: quota of the l-th level = ceil(tau_l * visible blocks),
+        # with tau_l at the float32 value the C interface carries, in exact
+        # rational arithmetic
+        quota = [math.ceil(Fraction(struct.unpack("f", struct.pack("f", t))[0]) * len(vis))
+                 for t in tau]
+        for r, j in enumerate(ranked):
             lv = -1
             for l in range(4):
-                if c < tau[l]:
+                if (r < quota[l]) if rule == "quantile" else (c < tau[l]):
                     lv = l
                     break
             levels[a][j] = lv

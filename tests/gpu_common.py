@@ -37,7 +37,8 @@ def params_for(w: W.Workload, tau=None) -> P.Params:
     return P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk,
                          W.thresholds(w) if tau is None else tau, w.causal,
                          w.forced_prefix_tokens, 0.0,
-                         torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+                         torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                         P.ASSIGN_QUANTILE if w.assign == "quantile" else P.ASSIGN_THRESHOLD)
 
 
 @dataclass
@@ -92,12 +93,15 @@ def oracle_heads(w: W.Workload, inp: W.Inputs, heads, tau=None, level_map=None):
         V = inp.as_f64("v", b, h // grp)
         res[(b, h)] = O.psa_head(Q, K, V, w.q_blk, w.kv_blk, tau, w.causal,
                                  w.forced_prefix_tokens, None,
-                                 None if level_map is None else level_map[b, h])
+                                 None if level_map is None else level_map[b, h], rule=w.assign)
     return res
 
 
-def map_mismatch_report(gpu_map: np.ndarray, mask: O.MaskResult, tau: Sequence[float]):
-    """Counts (unexplained, near_threshold, near_tie) mismatches of one head's map."""
+def map_mismatch_report(gpu_map: np.ndarray, mask: O.MaskResult, tau: Sequence[float],
+                        rule: str = "threshold"):
+    """Counts (unexplained, near_threshold, near_tie) mismatches of one head's map.
+    Under the quantile rule levels follow ranks only, so no mismatch is
+    excused by a running mass near a threshold; near-ties still are."""
     om = mask.level_map
     unexplained = near_thr = near_tie = 0
     bad = np.argwhere(gpu_map != om)
@@ -105,7 +109,7 @@ def map_mismatch_report(gpu_map: np.ndarray, mask: O.MaskResult, tau: Sequence[f
         g, o = int(gpu_map[a, j]), int(om[a, j])
         lo, hi = sorted((4 if g < 0 else g, 4 if o < 0 else o))
         c = mask.cum_before[a, j]
-        if any(abs(c - tau[l]) < MAP_EPS_C for l in range(lo, min(hi, 4))):
+        if rule == "threshold" and any(abs(c - tau[l]) < MAP_EPS_C for l in range(lo, min(hi, 4))):
             near_thr += 1
             continue
         pj = mask.mass[a, j]

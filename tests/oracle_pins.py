@@ -174,6 +174,68 @@ def pin_causal_overrides(O):
     assert r2.level_map[:, 0].tolist() == [0, 0] and r2.level_map[:, 1].tolist() == [0, 0]
 
 
+def pin_assign_quantile_handmade(O):
+    """Hand-worked quantile-rule assignments
+    (tests/golden/assign_levels_quantile_handmade.json)."""
+    with open(os.path.join(GOLDEN, "assign_levels_quantile_handmade.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        P = np.array(c["P"], dtype=np.float64)
+        z = np.log(P)[None, :]
+        r = O.assign_levels(z, c["tau"], N=64 * len(P), bq=64, bk=64, rule="quantile")
+        assert r.level_map[0].tolist() == c["levels"], (c["name"], r.level_map[0].tolist())
+
+
+def pin_assign_quantile_counts(O):
+    """Quantile rule, non-causal rows with no overrides: level l holds exactly
+    ceil(t_l n) - ceil(t_(l-1) n) blocks (t = the float32 tau, worked here in
+    exact rational arithmetic), and they are the next-heaviest blocks."""
+    from fractions import Fraction
+    rng = np.random.default_rng(7)
+    n = 37
+    z = rng.standard_normal((5, n)) * 2.0
+    tau = (0.1, 0.3, 0.55, 0.8)
+    r = O.assign_levels(z, tau, N=64 * n, bq=64, bk=64, rule="quantile")
+    K = [math.ceil(Fraction(float(np.float32(t))) * n) for t in tau]
+    for a in range(5):
+        row = r.level_map[a]
+        prev = 0
+        for l in range(4):
+            assert int((row == l).sum()) == K[l] - prev
+            prev = K[l]
+        assert int((row == -1).sum()) == n - K[3]
+        # heavier blocks never get a higher level than lighter ones
+        order = np.argsort(-z[a], kind="stable")
+        lv = np.where(row[order] < 0, 4, row[order])
+        assert np.all(np.diff(lv) >= 0)
+
+
+def pin_assign_quantile_permutation_and_causal(O):
+    """Quantile rule: shuffling the KV blocks shuffles the map the same way;
+    causal rows take their quotas of their own visible blocks."""
+    rng = np.random.default_rng(8)
+    z = rng.standard_normal((3, 40)) * 2.0
+    tau = (0.25, 0.5, 0.75, 0.875)
+    base = O.assign_levels(z, tau, N=64 * 40, bq=64, bk=64, rule="quantile").level_map
+    perm = rng.permutation(40)
+    shuf = O.assign_levels(z[:, perm], tau, N=64 * 40, bq=64, bk=64, rule="quantile").level_map
+    assert np.array_equal(shuf, base[:, perm])
+    # causal, N = 1024, 128-row query blocks: query block 3 sees KV blocks 0..7
+    zc = rng.standard_normal((8, 16))
+    rc = O.assign_levels(zc, tau, N=1024, bq=128, bk=64, causal=True, rule="quantile")
+    row = rc.level_map[3]
+    assert np.all(row[8:] == -1)
+    # blocks 6, 7 straddle the diagonal (level 0); the rest follow quotas of 8
+    assert row[6] == 0 and row[7] == 0
+    vis_rank = np.argsort(-zc[3, :8], kind="stable")
+    K = [2, 4, 6, 7]                                   # ceil(8 * tau)
+    for rnk, j in enumerate(vis_rank):
+        if j in (6, 7):
+            continue
+        want = next((l for l in range(4) if rnk < K[l]), -1)
+        assert row[j] == want, (j, rnk, row[j], want)
+
+
 # --------------------------------------------------------------- attention
 
 def _rand_head(seed, N, d):

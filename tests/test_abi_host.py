@@ -92,6 +92,13 @@ def test_selftest_argument_errors_before_any_launch():
     assert P.lib().psa_selftest_wait_timeout(ctypes.byref(bad), B, need, 1000, None) == 1
 
 
+def test_assign_rule_validated():
+    p = P.make_params(1, 2, 2, 1024, 64, assign=P.ASSIGN_QUANTILE)
+    assert P.workspace_size(p) > 0
+    p.assign = 2
+    assert P.workspace_size(p) == 0                                   # unknown rule
+
+
 def test_status_strings():
     for s in range(7):
         assert P.status_string(s)

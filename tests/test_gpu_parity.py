@@ -45,6 +45,23 @@ CASES = {
     "bf16_full_sort": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0,
                                        grid=(1, 47, 203), coarse=(1, 12, 51),
                                        forced_prefix_tokens=0, seed=18, target="alpha:1.0"),
+    # quantile rule (per-level quotas of blocks by rank): 16 blocks per row,
+    # one per lane, with fractional quotas
+    "f32_tiny_quantile": W.with_overrides(BASE["tiny_f32"], assign="quantile", seed=19),
+    # quantile rule through the candidate cut (K_3 = 23 of 150), text prefix forced
+    "bf16_quantile_cut": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=226,
+                                          grid=(1, 42, 222), coarse=(1, 11, 56),
+                                          forced_prefix_tokens=226, seed=20, target="alpha:0.15",
+                                          assign="quantile"),
+    # quantile rule, causal with grouped queries (quotas of each row's visible blocks)
+    "bf16_quantile_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 47, 203),
+                                             coarse=(1, 12, 51), seed=21, target="alpha:0.3",
+                                             assign="quantile"),
+    # quantile rule with tau_3 = 1: every visible block kept, the full sort
+    "bf16_quantile_full": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0,
+                                           grid=(1, 47, 203), coarse=(1, 12, 51),
+                                           forced_prefix_tokens=0, seed=22, target="alpha:1.0",
+                                           assign="quantile"),
 }
 
 _cache = {}
@@ -116,7 +133,7 @@ def test_level_map(name):
     gm = run.level_map.cpu().numpy()
     tau = W.thresholds(w)
     for (b, h), r in ref.items():
-        unexplained, thr, tie = G.map_mismatch_report(gm[b, h], r.mask, tau)
+        unexplained, thr, tie = G.map_mismatch_report(gm[b, h], r.mask, tau, w.assign)
         assert unexplained == 0, (b, h, unexplained, thr, tie)
         mass = G.to_f64(run.mass[b, h])
         assert np.abs(mass - r.mask.mass).max() <= 1e-5
@@ -190,11 +207,31 @@ def test_fused_forward(name):
     gm = run.level_map.cpu().numpy()
     tau = W.thresholds(w)
     for (b, h), r in ref.items():
-        assert G.map_mismatch_report(gm[b, h], r.mask, tau)[0] == 0
+        assert G.map_mismatch_report(gm[b, h], r.mask, tau, w.assign)[0] == 0
     ref_g = G.oracle_heads(w, inp, list(ref), level_map=gm)
     gO = G.to_f64(run.O)
     for (b, h), r in ref_g.items():
         G.compare_out(gO[b, h], r.O, w.dtype)
+
+
+def test_quantile_long_rows_shared_memory_sort():
+    """Rows of more than 1024 KV blocks sort in shared memory: the quantile
+    rule there (one head, N = 66000: 1032 blocks per row), the map only."""
+    w = W.with_overrides(BASE["cogvideox_5b"], Hq=1, Hkv=1, n_text=0, grid=(4, 110, 150),
+                         coarse=(1, 28, 38), forced_prefix_tokens=0, seed=23,
+                         target="alpha:0.2", assign="quantile")
+    assert w.Nk == 1032
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp)
+    gm = run.level_map.cpu().numpy()[0, 0]
+    Q, K = inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0)
+    pyr = O.build_pyramid(K, K)
+    z = O.block_logits(O.query_block_means(Q, w.q_blk), pyr, w.kv_blk, 1.0 / np.sqrt(w.d))
+    mask = O.assign_levels(z, W.thresholds(w), w.N, w.q_blk, w.kv_blk, w.causal, 0, "quantile")
+    assert G.map_mismatch_report(gm, mask, W.thresholds(w), "quantile")[0] == 0
+    # every row keeps exactly K_3 blocks
+    K3 = O.quotas(w.Nk, W.thresholds(w))[3]
+    assert np.all((gm >= 0).sum(-1) == K3)
 
 
 def test_no_device_timeouts_recorded():

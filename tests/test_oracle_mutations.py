@@ -31,6 +31,10 @@ MUTATIONS = {
     "straddle test shifted": ("np.minimum((j + 1) * bk, N) - 1 >= q_lo", "np.minimum((j + 1) * bk, N) - 1 > q_lo + 63"),
     "forced prefix ignored": ("row[strad | forced] = 0", "row[strad] = 0"),
     "values pooled from keys": ("values[l], _ = pool_tokens(V, f)", "values[l], _ = pool_tokens(K, f)"),
+    "quantile quotas rounded down": ("np.ceil(t * float(n_visible))", "np.floor(t * float(n_visible))"),
+    "quantile tau in double": ("np.asarray(tau, dtype=np.float32).astype(np.float64)", "np.asarray(tau, dtype=np.float64)"),
+    "quantile rank <= quota": ("out[rank < K[l]] = l", "out[rank <= K[l]] = l"),
+    "quantile quotas of all blocks": ("quotas(len(order), tau)", "quotas(Nk, tau)"),
 }
 
 
@@ -49,12 +53,16 @@ def _mutant(old, new):
 
 def _bruteforce_agrees(M):
     rng = np.random.default_rng(21)
-    for N, d, bq, causal, forced in ((203, 8, 64, False, 70), (187, 4, 64, True, 0),
-                                     (509, 8, 64, False, 0)):
+    for N, d, bq, causal, forced, rule in ((203, 8, 64, False, 70, "threshold"),
+                                           (187, 4, 64, True, 0, "threshold"),
+                                           (509, 8, 64, False, 0, "threshold"),
+                                           (509, 8, 64, False, 0, "quantile"),
+                                           (701, 4, 64, True, 0, "quantile")):
         Q, K, V = (rng.standard_normal((N, d)) * 1.5 for _ in range(3))
-        tau = (0.5, 0.7, 0.85, 0.95)
-        O_b, _, lv = psa_bruteforce(Q.tolist(), K.tolist(), V.tolist(), bq, 64, tau, causal, forced)
-        r = M.psa_head(Q, K, V, bq, 64, tau, causal, forced)
+        tau = (0.5, 0.7, 0.85, 0.95) if rule == "threshold" else (0.15, 0.3, 0.5, 0.7)
+        O_b, _, lv = psa_bruteforce(Q.tolist(), K.tolist(), V.tolist(), bq, 64, tau, causal, forced,
+                                    rule=rule)
+        r = M.psa_head(Q, K, V, bq, 64, tau, causal, forced, rule=rule)
         if r.mask.level_map.tolist() != lv or not np.allclose(r.O, np.array(O_b), atol=1e-10):
             return False
     return True
@@ -74,6 +82,7 @@ def test_mutation_is_caught_by_a_pin(name):
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught_by_bruteforce(name):
-    if name in ("threshold <= instead of <", "ties to the higher index"):
-        pytest.skip("random masses never tie or land on a threshold; the golden cases pin these")
+    if name in ("threshold <= instead of <", "ties to the higher index", "quantile tau in double"):
+        pytest.skip("random masses never tie or land on a threshold, and these quotas are exact "
+                    "in both precisions; the golden cases pin these")
     assert not _bruteforce_agrees(_mutant(*MUTATIONS[name]))

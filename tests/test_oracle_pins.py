@@ -15,16 +15,17 @@ def test_pin(pin):
     pin(O)
 
 
+@pytest.mark.parametrize("rule", ["threshold", "quantile"])
 @pytest.mark.parametrize("N,d,bq,causal,forced", [
     (256, 8, 64, False, 0), (200, 8, 64, False, 70), (256, 4, 128, True, 0),
     (184, 8, 64, True, 0), (64, 8, 64, False, 0), (9, 4, 64, False, 0)])
-def test_bruteforce_matches_oracle(N, d, bq, causal, forced):
+def test_bruteforce_matches_oracle(N, d, bq, causal, forced, rule):
     rng = np.random.default_rng(N + d)
     Q, K, V = (rng.standard_normal((N, d)) * 1.5 for _ in range(3))
-    tau = (0.5, 0.7, 0.85, 0.95)
+    tau = (0.5, 0.7, 0.85, 0.95) if rule == "threshold" else (0.2, 0.4, 0.6, 0.8)
     O_b, lse_b, lv_b = psa_bruteforce(Q.tolist(), K.tolist(), V.tolist(), bq, 64, tau,
-                                      causal, forced)
-    r = O.psa_head(Q, K, V, bq, 64, tau, causal, forced)
+                                      causal, forced, rule=rule)
+    r = O.psa_head(Q, K, V, bq, 64, tau, causal, forced, rule=rule)
     assert r.mask.level_map.tolist() == lv_b
     assert np.allclose(r.O, np.array(O_b), atol=1e-12)
     assert np.allclose(r.lse, np.array(lse_b), atol=1e-12)

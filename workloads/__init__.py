@@ -58,6 +58,7 @@ class Workload:
     seed: int
     target: str                     # how tau is chosen: "fixed", "alpha:0.15", "skip:0.91", "keep:0.35"
     pool: Tuple[int, int, int, int] = (1, 2, 4, 8)
+    assign: str = "threshold"       # level assignment rule: "threshold" or "quantile"
 
     @property
     def N(self) -> int:
