@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: run only this many query heads (KV heads scaled to match)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="batch: every rank runs its own batch (weak scaling, the default); "
+                         "heads: the ranks split the heads of one problem (strong scaling)")
     return ap.parse_args()
 
 
@@ -258,10 +261,20 @@ def run_ours(args, rank, world, local_rank):
     if args.heads:
         grp = w.Hq // w.Hkv
         w = W.with_overrides(w, Hq=args.heads, Hkv=max(1, args.heads // grp))
+    w_job = w                                 # the whole job's problem
+    if args.shard == "heads":
+        # strong scaling: this rank's heads of one problem (its own slice of
+        # the generator's heads; the shards need no exchange)
+        q0, q1, kv0, kv1 = P.head_shard(w.Hq, w.Hkv, rank, world)
+        full = W.make_inputs(w, heads_q=list(range(q0, q1)), heads_kv=list(range(kv0, kv1)))
+        w = W.with_overrides(w, Hq=q1 - q0, Hkv=kv1 - kv0)
+        inp = W.Inputs(w, np.ascontiguousarray(full.q[:, q0:q1]),
+                       np.ascontiguousarray(full.k[:, kv0:kv1]), np.ascontiguousarray(full.v[:, kv0:kv1]))
+    else:
+        inp = W.make_inputs(w, batch0=rank_batch0(rank, w.B))
     p = P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk, tau, w.causal,
                       w.forced_prefix_tokens, 0.0,
                       torch.bfloat16 if w.dtype == "bf16" else torch.float32)
-    inp = W.make_inputs(w, batch0=rank_batch0(rank, w.B))
 
     def host(x):
         t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
@@ -321,7 +334,10 @@ def run_ours(args, rank, world, local_rank):
     mask_ms = [e[1].elapsed_time(e[2]) for e in ev]
     attn_ms = [e[2].elapsed_time(e[3]) for e in ev]
     ms = max_over_ranks(sum(step_ms), world, dev) / args.steps
-    value = whole_job_tflops(dense, world, ms)
+    # weak: every rank's batch has the workload's dense FLOPs; strong: the
+    # ranks' shares add up to one problem's
+    value = (whole_job_tflops(dense, world, ms) if args.shard == "batch"
+             else w_job.dense_flops() / (ms * 1e-3) / 1e12)
 
     # end to end through the public API with host buffers: H2D of Q, K, V, the
     # forward, D2H of O, every step inside the timed region
@@ -339,6 +355,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    job_dense = dense * world if args.shard == "batch" else w_job.dense_flops()
     P.check_device(p, ws)
 
     bf16_peak, hbm_peak, peak_kind = peaks()
@@ -359,16 +376,19 @@ def run_ours(args, rank, world, local_rank):
         parity = sampled_parity(w, results, lm, out)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak" if args.shard == "batch" else "strong",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded smooth 3-D field + noise)",
-        "config": {"workload": w.name, "global_batch": w.B * world, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+        "config": {"workload": w.name, "global_batch": w.B * world if args.shard == "batch" else w.B,
+                   "shard": args.shard, "B": w.B, "Hq": w_job.Hq, "Hkv": w_job.Hkv, "N": w.N, "d": w.d,
                    "q_blk": w.q_blk, "kv_blk": w.kv_blk, "tau": [round(t, 6) for t in tau],
                    "causal": w.causal, "skipped_dense_fraction": 1.0 - executed / dense,
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
-                   "parallelism": f"independent batch per GPU x{world}"},
+                   "parallelism": (f"independent batch per GPU x{world}" if args.shard == "batch"
+                                   else f"heads of one problem split over {world} GPUs")},
         "ms_per_call": ms, "pct_bf16_peak_dense_equiv": 100.0 * value / world / bf16_peak,
-        "executed_tflops": executed * world / (ms * 1e-3) / 1e12,
+        "executed_tflops": executed * (world if args.shard == "batch" else 1) / (ms * 1e-3) / 1e12,
         "kernel_ms": {"pyramid": pyr_avg, "mask": mask_avg, "attention": attn_avg},
         "hbm": {"peak_gbs": hbm_peak, "peak_kind": f"{peak_kind} copy",
                 "pyramid": {"bytes": pyramid_bytes(w), "gbs": pyr_gbs, "frac": pyr_gbs / hbm_peak},
@@ -381,7 +401,7 @@ def run_ours(args, rank, world, local_rank):
                      "padding_fraction": 1.0 - (keys_per_row.sum() / max(padded_keys, 1.0))},
         "cpu_baseline": cpu,
         "parity": parity,
-        "e2e": {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": job_dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * es),
                 "d2h_bytes_per_step": int(out.numel() * es)},

@@ -19,8 +19,9 @@
  *    the one call that waits on the stream).  All work is enqueued on `stream`
  *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
  *  - Tensors are dense row-major: Q/O [B, Hq, N, d], K/V [B, Hkv, N, d] with d
- *    contiguous; element type is params->dtype (fp32 or bf16).  Device
- *    pointers must be 16-byte aligned.
+ *    contiguous; element type is params->dtype (fp32 or bf16).  Q, K, V and O
+ *    must be 16-byte aligned; lse and block_mass, written one float at a
+ *    time, 4-byte aligned; the workspace 256-byte aligned.
  *  - Arguments are validated on the host before anything is launched; on an
  *    error nothing is enqueued and a psa_status_t other than PSA_OK returns.
  *    A CUDA launch error is returned as PSA_ERR_CUDA.
@@ -42,7 +43,7 @@ typedef enum {
   PSA_OK = 0,
   PSA_ERR_INVALID_ARG = 1,          /* NULL pointer, bad size, tau not monotone, ... */
   PSA_ERR_UNSUPPORTED = 2,          /* valid but not implemented (e.g. d = 96)        */
-  PSA_ERR_MISALIGNED = 3,           /* a device pointer is not 16-byte aligned         */
+  PSA_ERR_MISALIGNED = 3,           /* a device pointer breaks its alignment rule       */
   PSA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < psa_workspace_size(params)    */
   PSA_ERR_CUDA = 5,                 /* a CUDA call or launch failed                    */
   PSA_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up waiting (see psa_check_device) */

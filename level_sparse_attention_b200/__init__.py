@@ -178,19 +178,68 @@ def map_shape(p: Params) -> Tuple[int, int, int, int]:
 def psa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_blk: int = 128,
                 kv_blk: int = 64, tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97),
                 causal: bool = False, forced_prefix_tokens: int = 0, scale: float = 0.0,
-                return_map: bool = False, workspace: Optional[torch.Tensor] = None):
+                return_map: bool = False, workspace: Optional[torch.Tensor] = None,
+                assign: int = ASSIGN_THRESHOLD):
     """PSA forward on CUDA tensors q [B, Hq, N, d], k/v [B, Hkv, N, d]
     (contiguous, bf16 or fp32).  Returns (O, lse) or (O, lse, level_map)."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     p = make_params(B, Hq, Hkv, N, d, q_blk, kv_blk, tau, causal, forced_prefix_tokens, scale,
-                    q.dtype)
+                    q.dtype, assign)
     ws = workspace if workspace is not None else new_workspace(p, q.device)
     O = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     lm = torch.empty(map_shape(p), dtype=torch.int8, device=q.device) if return_map else None
     forward(p, q.contiguous(), k.contiguous(), v.contiguous(), O, ws, lse, lm)
     return (O, lse, lm) if return_map else (O, lse)
+
+
+def head_shard(Hq: int, Hkv: int, rank: int, world: int) -> Tuple[int, int, int, int]:
+    """The heads rank `rank` of `world` takes of one problem: query heads
+    [q0, q1) and the KV heads [kv0, kv1) they read (query head h reads KV
+    head h // (Hq / Hkv)).  Every (batch, head) of the forward pass is
+    independent, so the shards need no exchange.  With at least as many KV
+    heads as ranks, ranks take whole groups of query heads sharing a KV head
+    (as even a split of the KV heads as possible); with fewer, each KV head's
+    group is split among world / Hkv ranks, so a shard never straddles two
+    groups.  Either way the shard's own grouping matches the global one.
+    Returns (q0, q1, kv0, kv1); raises ValueError for a split it cannot make."""
+    if Hq <= 0 or Hkv <= 0 or Hq % Hkv or not 0 <= rank < world:
+        raise ValueError("bad head counts or rank")
+    G = Hq // Hkv
+    if Hkv >= world:
+        kv0, kv1 = rank * Hkv // world, (rank + 1) * Hkv // world
+        return kv0 * G, kv1 * G, kv0, kv1
+    if world % Hkv:
+        raise ValueError(f"{world} ranks cannot split {Hkv} KV heads' groups evenly")
+    per = world // Hkv                       # ranks per KV head
+    if per > G:
+        raise ValueError(f"{per} ranks per KV head exceed its {G} query heads")
+    kv = rank // per
+    i = rank % per
+    q0, q1 = kv * G + i * G // per, kv * G + (i + 1) * G // per
+    return q0, q1, kv, kv + 1
+
+
+def psa_forward_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                      lse: Optional[torch.Tensor], p: Params, rank: int, world: int,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> Params:
+    """This rank's share of one forward pass: the heads of head_shard for
+    every batch element, written into the matching heads of `out` (and
+    `lse`).  q, k, v, out: [B, H, N, d] contiguous device tensors of the full
+    problem described by `p`; every rank may hold them whole (they are read
+    and written only at its heads).  One psa_forward call per batch element on
+    the contiguous head slices.  Returns the per-call params."""
+    q0, q1, kv0, kv1 = head_shard(p.Hq, p.Hkv, rank, world)
+    sp = Params.from_buffer_copy(p)
+    sp.B, sp.Hq, sp.Hkv = 1, q1 - q0, kv1 - kv0
+    if sp.Hq == 0:
+        return sp
+    ws = workspace if workspace is not None else new_workspace(sp, q.device)
+    for b in range(p.B):
+        forward(sp, q[b, q0:q1], k[b, kv0:kv1], v[b, kv0:kv1], out[b, q0:q1], ws,
+                None if lse is None else lse[b, q0:q1], None, stream)
+    return sp
 
 
 def workspace_layout(p: Params) -> dict:

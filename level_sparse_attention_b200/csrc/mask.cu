@@ -245,8 +245,13 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[K]) {
 constexpr int kCandPerLane = 4;
 constexpr int kCand = 32 * kCandPerLane;
 
+// Rows of more than 1024 blocks keep their keys in shared memory; their
+// candidate set holds up to kCandS blocks, kCandPerLaneS per lane.
+constexpr int kCandPerLaneS = 8;
+constexpr int kCandS = 32 * kCandPerLaneS;
+
 __host__ __device__ inline size_t assign_key_bytes(int K, int n2) {
-  return K == 0 ? (size_t)n2 * 8 : (K > kCandPerLane ? (size_t)kCand * 8 : 0);
+  return K == 0 ? (size_t)(n2 + kCandS) * 8 : (K > kCandPerLane ? (size_t)kCand * 8 : 0);
 }
 
 // The level of a visible block from its place in the ranking.  Threshold
@@ -467,6 +472,100 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   } else {
     for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
     __syncwarp();
+    // Candidate cut, as in the register path, over the keys in shared memory
+    // (lane L reads keys L, L + 32, ...): blocks with P >= t are a prefix of
+    // the ranking; t is bisected until they reach past every kept rank and
+    // number at most kCandS, and only they are ranked.
+    bool done = false;
+    unsigned long long* cand = key + n2;
+    const float target = a.tau[kLevels - 1] + 1e-3f;
+    const int kq = rule.quota[kLevels - 1];
+    if (rule.quantile ? kq <= kCandS : target <= 0.99f) {
+      auto pk = [](unsigned long long k) { return __uint_as_float((unsigned)(k >> 32)); };
+      auto enough = [&](float t, int* cnt) {
+        float m = 0.f;
+        int c = 0;
+        for (int i = lane; i < nvis; i += 32) {
+          const float pi = pk(key[i]);
+          const bool in = pi >= t;
+          m += in ? pi : 0.f;
+          c += in;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          m += __shfl_xor_sync(0xffffffffu, m, o);
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+        }
+        *cnt = c;
+        return rule.quantile ? c >= kq : m >= target;
+      };
+      float pmax = 0.f;
+      for (int i = lane; i < nvis; i += 32) pmax = fmaxf(pmax, pk(key[i]));
+      pmax = warp_max(pmax);
+      int m_hi, m;
+      float lo = 0.f, hi = pmax, t;
+      if (enough(hi, &m_hi)) {
+        t = hi;
+        m = m_hi;
+      } else {
+        int m_lo = nvis;
+        for (int it = 0; it < 40 && m_lo > kCandS; ++it) {
+          const float mid = 0.5f * (lo + hi);
+          if (!(mid > lo && mid < hi)) break;
+          int c;
+          if (enough(mid, &c)) {
+            lo = mid;
+            m_lo = c;
+          } else {
+            hi = mid;
+          }
+        }
+        t = lo;
+        m = m_lo;
+      }
+      if (m <= kCandS) {
+        // compact the candidates (in index order; the ranking below needs no order)
+        int base = 0;
+        for (int i0 = 0; i0 < nvis; i0 += 32) {
+          const int i = i0 + lane;
+          const unsigned long long ki = i < nvis ? key[i] : 0ull;
+          const bool in = i < nvis && pk(ki) >= t;
+          const unsigned bal = __ballot_sync(0xffffffffu, in);
+          if (in) cand[base + __popc(bal & ((1u << lane) - 1))] = ki;
+          base += __popc(bal);
+        }
+        __syncwarp();
+        unsigned long long mk[kCandPerLaneS];
+        float c[kCandPerLaneS];
+        int rk[kCandPerLaneS];
+#pragma unroll
+        for (int r = 0; r < kCandPerLaneS; ++r) {
+          const int i = lane + 32 * r;
+          mk[r] = i < m ? cand[i] : ~0ull;
+          c[r] = 0.f;
+          rk[r] = 0;
+        }
+        for (int jj = 0; jj < m; ++jj) {
+          const unsigned long long kj = cand[jj];           // same address in every lane
+          const float pj_ = pk(kj);
+#pragma unroll
+          for (int r = 0; r < kCandPerLaneS; ++r) {
+            const bool before = kj > mk[r];
+            c[r] += before ? pj_ : 0.f;
+            rk[r] += before;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < kCandPerLaneS; ++r) {
+          if (lane + 32 * r < m) {
+            const int j = (int)(0xffffffffu - (unsigned)(mk[r] & 0xffffffffu));
+            lev[j] = rule.level(c[r], rk[r]);
+          }
+        }
+        done = true;
+      }
+    }
+    if (!done) {
     // bitonic sort in shared memory, descending: P high, then lower index first
     for (int k = 2; k <= n2; k <<= 1) {
       for (int sd = k >> 1; sd > 0; sd >>= 1) {
@@ -492,6 +591,7 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
       const int j = (int)(0xffffffffu - (unsigned)(key[r] & 0xffffffffu));
       lev[j] = rule.level(c, r);
       c += pr;
+    }
     }
   }
   __syncwarp();

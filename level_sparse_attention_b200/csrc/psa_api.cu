@@ -9,6 +9,8 @@ namespace psa {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// lse and block_mass are written one float at a time
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 psa_status_t validate(const psa_params_t* p) {
   if (!p) return PSA_ERR_INVALID_ARG;
@@ -115,7 +117,7 @@ psa_status_t psa_score_and_mask(const psa_params_t* params, const void* Q, void*
   Layout L;
   if ((r = check_ws(params, workspace, workspace_bytes, &L)) != PSA_OK) return r;
   if ((r = check_ptrs({Q})) != PSA_OK) return r;
-  if (block_mass && !aligned16(block_mass)) return PSA_ERR_MISALIGNED;
+  if (block_mass && !aligned4(block_mass)) return PSA_ERR_MISALIGNED;
   return run_mask(params, L, Q, workspace, level_map, block_mass, (cudaStream_t)stream);
 }
 
@@ -127,7 +129,7 @@ psa_status_t psa_attention_fwd(const psa_params_t* params, const void* Q, const 
   Layout L;
   if ((r = check_ws(params, workspace, workspace_bytes, &L)) != PSA_OK) return r;
   if ((r = check_ptrs({Q, K, V, O})) != PSA_OK) return r;
-  if (lse && !aligned16(lse)) return PSA_ERR_MISALIGNED;
+  if (lse && !aligned4(lse)) return PSA_ERR_MISALIGNED;
   return run_attention(params, L, Q, K, V, workspace, level_map, O, lse, (cudaStream_t)stream);
 }
 
@@ -139,7 +141,7 @@ psa_status_t psa_forward(const psa_params_t* params, const void* Q, const void* 
   Layout L;
   if ((r = check_ws(params, workspace, workspace_bytes, &L)) != PSA_OK) return r;
   if ((r = check_ptrs({Q, K, V, O})) != PSA_OK) return r;
-  if (lse && !aligned16(lse)) return PSA_ERR_MISALIGNED;
+  if (lse && !aligned4(lse)) return PSA_ERR_MISALIGNED;
   cudaStream_t st = (cudaStream_t)stream;
   if ((r = run_pyramid(params, L, K, V, workspace, st)) != PSA_OK) return r;
   if ((r = run_mask(params, L, Q, workspace, level_map, nullptr, st)) != PSA_OK) return r;
@@ -171,7 +173,7 @@ const char* psa_status_string(psa_status_t status) {
     case PSA_OK: return "ok";
     case PSA_ERR_INVALID_ARG: return "invalid argument";
     case PSA_ERR_UNSUPPORTED: return "unsupported configuration";
-    case PSA_ERR_MISALIGNED: return "device pointer not 16-byte aligned (workspace: 256-byte)";
+    case PSA_ERR_MISALIGNED: return "device pointer misaligned (Q/K/V/O 16-byte, lse/mass 4-byte, workspace 256-byte)";
     case PSA_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than psa_workspace_size()";
     case PSA_ERR_CUDA: return "CUDA error";
     case PSA_ERR_DEVICE_TIMEOUT: return "a kernel gave up waiting on the device (timeout)";

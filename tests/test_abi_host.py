@@ -73,8 +73,10 @@ def test_argument_errors_before_any_launch():
     bad = P.make_params(1, 2, 2, 1024, 96)
     assert _call_forward(bad, A, A, A, A, B, need) == 2             # d = 96 unsupported
     assert P.lib().psa_build_pyramid(ctypes.byref(p), None, A, B, need, None) == 1
-    assert P.lib().psa_score_and_mask(ctypes.byref(p), A, B, need, None, mis, None) == 3
-    assert P.lib().psa_attention_fwd(ctypes.byref(p), A, A, A, B, need, None, A, mis, None) == 3
+    mis4 = ctypes.c_void_p(0x10002)         # lse and block_mass need float (4-byte) alignment
+    assert P.lib().psa_score_and_mask(ctypes.byref(p), A, B, need, None, mis4, None) == 3
+    assert P.lib().psa_attention_fwd(ctypes.byref(p), A, A, A, B, need, None, A, mis4, None) == 3
+    assert P.lib().psa_forward(ctypes.byref(p), A, A, A, A, mis4, None, B, need, None) == 3
 
 
 def test_selftest_argument_errors_before_any_launch():

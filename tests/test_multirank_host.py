@@ -57,6 +57,17 @@ def _rank_main(rank, world, port, out_dir):
         res = O.psa_head(inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0), inp.as_f64("v", 0, 0),
                          w.q_blk, w.kv_blk, W.thresholds(w), w.causal, w.forced_prefix_tokens)
 
+        # head sharding of one problem: this rank's heads through the oracle
+        wh = W.with_overrides(W.BY_NAME["tiny_f32"], Hq=4, Hkv=2, seed=3)
+        hi = W.make_inputs(wh)
+        import level_sparse_attention_b200 as PB
+        q0, q1, kv0, kv1 = PB.head_shard(wh.Hq, wh.Hkv, rank, world)
+        grp = wh.Hq // wh.Hkv
+        shard_out = np.stack([
+            O.psa_head(hi.as_f64("q", 0, h), hi.as_f64("k", 0, h // grp), hi.as_f64("v", 0, h // grp),
+                       wh.q_blk, wh.kv_blk, W.thresholds(wh)).O for h in range(q0, q1)])
+        assert all(kv0 <= h // grp < kv1 for h in range(q0, q1))
+
         # the reference arm returns without work on rank != 0
         class A:
             workload, steps, warmup, gpus = "tiny_f32", 1, 0, world
@@ -65,7 +76,7 @@ def _rank_main(rank, world, port, out_dir):
         dist.barrier()
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), ms=ms, tflops=tflops, b0=b0,
                  q=inp.q, out=res.O, lse=res.lse, level_map=res.mask.level_map,
-                 ref_none=ref is None)
+                 ref_none=ref is None, shard=np.array([q0, q1]), shard_out=shard_out)
     finally:
         dist.destroy_process_group()
 
@@ -109,3 +120,45 @@ def test_sharded_oracle_equals_global_batch(rank_results):
 
 def test_reference_arm_idles_off_rank_zero(rank_results):
     assert bool(rank_results[1]["ref_none"])
+
+
+def test_head_shards_together_equal_the_whole_problem(rank_results):
+    import oracle as O
+    import workloads as W
+    wh = W.with_overrides(W.BY_NAME["tiny_f32"], Hq=4, Hkv=2, seed=3)
+    hi = W.make_inputs(wh)
+    shards = sorted((tuple(r["shard"]), r["shard_out"]) for r in rank_results)
+    assert [s[0] for s in shards] == [(0, 2), (2, 4)]
+    got = np.concatenate([s[1] for s in shards])
+    for h in range(wh.Hq):
+        ref = O.psa_head(hi.as_f64("q", 0, h), hi.as_f64("k", 0, h // 2), hi.as_f64("v", 0, h // 2),
+                         wh.q_blk, wh.kv_blk, W.thresholds(wh)).O
+        np.testing.assert_array_equal(got[h], ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv,world", [(40, 40, 8), (12, 12, 5), (28, 4, 8), (28, 4, 4),
+                                          (48, 48, 3), (4, 2, 4), (8, 1, 2), (8, 1, 8), (6, 3, 1)])
+def test_head_shard_plan(Hq, Hkv, world):
+    import level_sparse_attention_b200 as PB
+    G = Hq // Hkv
+    got = [PB.head_shard(Hq, Hkv, r, world) for r in range(world)]
+    covered = []
+    for q0, q1, kv0, kv1 in got:
+        covered += list(range(q0, q1))
+        if q1 > q0:
+            # the shard's own grouping is the global one: local head i reads local
+            # KV head i // ((q1 - q0) / (kv1 - kv0)), global head q0 + i reads (q0 + i) // G
+            Gs = (q1 - q0) // (kv1 - kv0)
+            assert (q1 - q0) % (kv1 - kv0) == 0
+            assert all(kv0 + i // Gs == (q0 + i) // G for i in range(q1 - q0))
+    assert covered == list(range(Hq))                       # disjoint, in order, complete
+    sizes = [q1 - q0 for q0, q1, _, _ in got]
+    assert max(sizes) - min(sizes) <= G                     # balanced to within a group
+
+
+def test_head_shard_rejects_uneven_group_splits():
+    import level_sparse_attention_b200 as PB
+    with pytest.raises(ValueError):
+        PB.head_shard(28, 4, 0, 6)                          # 6 ranks, 4 KV heads
+    with pytest.raises(ValueError):
+        PB.head_shard(8, 1, 0, 16)                          # more ranks than query heads
