@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: run only this many query heads (KV heads scaled to match)")
+    ap.add_argument("--profile-kernels", action="store_true",
+                    help="after the timed region, run the steps again under the torch profiler "
+                         "(CUPTI) and add per-kernel microseconds to the line")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
                     help="batch: every rank runs its own batch (weak scaling, the default); "
                          "heads: the ranks split the heads of one problem (strong scaling)")
@@ -358,6 +361,22 @@ def run_ours(args, rank, world, local_rank):
     job_dense = dense * world if args.shard == "batch" else w_job.dense_flops()
     P.check_device(p, ws)
 
+    kernels_us = None
+    if args.profile_kernels:
+        # per-kernel device times over extra steps (not the timed ones)
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            for _ in range(args.steps):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
+        agg = {}
+        for e in prof.events():
+            if e.device_type == torch.autograd.DeviceType.CUDA and "psa::" in e.name:
+                name = e.name.split("(")[0].replace("void ", "").replace("psa::(anonymous namespace)::", "")
+                agg.setdefault(name, []).append(e.device_time_total)
+        kernels_us = {k: round(statistics.median(v), 2) for k, v in sorted(agg.items())}
+
     bf16_peak, hbm_peak, peak_kind = peaks()
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = executed / (attn_avg * 1e-3) / 1e12
@@ -406,6 +425,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * es),
                 "d2h_bytes_per_step": int(out.numel() * es)},
         "gpu_launches": 5 * args.steps,
+        "kernels_us": kernels_us,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -397,7 +397,11 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
           m = m_hi;
         } else {
           int m_lo = nvis;                 // the whole row: mass 1 >= target, nvis >= K_3
-          for (int it = 0; it < 40 && m_lo > kCand; ++it) {
+          // once the candidates fit, a few more steps shrink them (ranking
+          // costs m per candidate, a step one pass over the row)
+          int extra = 0;
+          for (int it = 0; it < 40; ++it) {
+            if (m_lo <= kCand && (m_lo <= 48 || extra++ >= 3)) break;
             const float mid = 0.5f * (lo + hi);
             if (!(mid > lo && mid < hi)) break;
             int c;
@@ -509,7 +513,9 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
         m = m_hi;
       } else {
         int m_lo = nvis;
-        for (int it = 0; it < 40 && m_lo > kCandS; ++it) {
+        int extra = 0;
+        for (int it = 0; it < 40; ++it) {
+          if (m_lo <= kCandS && (m_lo <= 48 || extra++ >= 6)) break;
           const float mid = 0.5f * (lo + hi);
           if (!(mid > lo && mid < hi)) break;
           int c;
