@@ -61,7 +61,7 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "2ee739a4de2f4460"): 471.842304e6 + 92.477952e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "27cc7203d4316d64"): 473.676032e6 + 93.238528e6}
 
 
 def attn_source_hash() -> str:
@@ -373,7 +373,8 @@ def run_ours(args, rank, world, local_rank):
         agg = {}
         for e in prof.events():
             if e.device_type == torch.autograd.DeviceType.CUDA and "psa::" in e.name:
-                name = e.name.split("(")[0].replace("void ", "").replace("psa::(anonymous namespace)::", "")
+                name = e.name.replace("psa::(anonymous namespace)::", "").replace("void ", "")
+                name = name.split("(")[0]
                 agg.setdefault(name, []).append(e.device_time_total)
         kernels_us = {k: round(statistics.median(v), 2) for k, v in sorted(agg.items())}
 
