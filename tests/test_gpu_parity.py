@@ -237,3 +237,42 @@ def test_quantile_long_rows_shared_memory_sort():
 def test_no_device_timeouts_recorded():
     w, inp, _, run = setup("bf16_d128")
     P.check_device(run.p, run.ws)
+
+
+@pytest.mark.parametrize("boost", [40.0, 600.0])
+def test_attention_logit_jumps_across_tiles(boost):
+    """A row's largest logits arrive on a later tile of its stream: keys of
+    some coarser-level blocks are set to `boost` along the query direction
+    (exact in bf16, and so are their pooled means), about +20 (boost 40: a
+    rescale deferred to the stream's next tile) or about +300 (boost 600: past
+    the direct-exponential range, so the tile half is redone after an
+    immediate rescale, after the tile's first half of P was stored) in log2
+    units.  External map: block j at level j // 8 (N = 2048, 32 blocks), so
+    each query block has 8 tiles; the boosted blocks 10, 11 and 14, 15 fill
+    the second halves of tiles 4 and 5 (one per stream), 30, 31 sit in tile 7."""
+    N, d, bq, bk = 2048, 128, 128, 64
+    rng = np.random.default_rng(41)
+    Q = rng.standard_normal((N, d)) * 0.1
+    Q[:, 0] += 4.0
+    K = rng.standard_normal((N, d)) * 0.1
+    V = rng.standard_normal((N, d))
+    for j in (10, 11, 14, 15, 30, 31):
+        K[j * bk:(j + 1) * bk, 0] = boost
+    to_bf16 = lambda x: W.bf16_bits_to_f32(W.f32_to_bf16_bits(x.astype(np.float32))).astype(np.float64)
+    Q, K, V = to_bf16(Q), to_bf16(K), to_bf16(V)
+    Nq, Nk = N // bq, N // bk
+    lm = np.repeat((np.arange(Nk) // 8).astype(np.int8)[None, :], Nq, axis=0)
+    p = P.make_params(1, 1, 1, N, d, bq, bk)
+    dev = lambda x: torch.from_numpy(W.f32_to_bf16_bits(x.astype(np.float32)).view(np.int16)) \
+        .view(torch.bfloat16).reshape(1, 1, N, d).cuda()
+    q, k, v = dev(Q), dev(K), dev(V)
+    ws = P.new_workspace(p)
+    out = torch.zeros_like(q)
+    lse = torch.zeros((1, 1, N), dtype=torch.float32, device="cuda")
+    P.build_pyramid(p, k, v, ws)
+    P.attention_fwd(p, q, k, v, ws, out, lse, torch.from_numpy(lm[None, None]).cuda())
+    torch.cuda.synchronize()
+    P.check_device(p, ws)
+    ref_O, ref_lse = O.pyramid_attention(Q, O.build_pyramid(K, V), lm, bq, bk, 1.0 / np.sqrt(d))
+    G.compare_out(G.to_f64(out[0, 0]), ref_O, "bf16")
+    G.compare_lse(lse[0, 0].cpu().numpy().astype(np.float64), ref_lse, "bf16")
