@@ -171,6 +171,34 @@ psa_status_t psa_forward_noalloc(const psa_params_t* params, const void* Q, cons
                                  const void* V, void* O, float* lse, int8_t* level_map,
                                  void* stream);
 
+/* psa_forward from host buffers, with the copies pipelined behind the
+ * kernels: the heads are split into `head_groups` groups (contiguous query
+ * heads with the KV heads they read: whole GQA groups when Hkv >= head_groups,
+ * else an even split of each KV head's query heads, which needs head_groups a
+ * multiple of Hkv), and for each batch element and group
+ *   - the group's Q and not-yet-copied K, V go host -> device on h2d_stream,
+ *   - the group's forward pass (psa_forward on the slices) runs on `stream`
+ *     once they have arrived,
+ *   - its O (and lse) go device -> host on d2h_stream,
+ * so one group's copies overlap another's kernels.  Every (batch, head) is
+ * independent, so the results equal one psa_forward over the whole problem.
+ *  Q_host, K_host, V_host, O_host, lse_host: host memory in the layout of
+ *    psa_forward (pinned memory lets the copies run asynchronously).
+ *  Q_dev, K_dev, V_dev, O_dev, lse_dev: device buffers for the whole problem,
+ *    aligned as for psa_forward; lse_host and lse_dev are both NULL or both
+ *    set.
+ *  workspace: psa_workspace_size(params) bytes (groups reuse it in turn).
+ *  stream, h2d_stream, d2h_stream: three distinct streams; everything is
+ *    enqueued, and `stream` completes only after the last copy to the host.
+ * Returns PSA_ERR_INVALID_ARG for bad parameters, a NULL buffer, streams that
+ * are not distinct or a group split that cannot be made; otherwise the status
+ * of the copies and of psa_forward. */
+psa_status_t psa_forward_host(const psa_params_t* params, const void* Q_host, const void* K_host,
+                              const void* V_host, void* O_host, float* lse_host, void* Q_dev,
+                              void* K_dev, void* V_dev, void* O_dev, float* lse_dev,
+                              void* workspace, size_t workspace_bytes, int head_groups,
+                              void* stream, void* h2d_stream, void* d2h_stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
  * check, PSA_ERR_CUDA if the stream reported an error, else PSA_OK. */

@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
             "psa_forward_noalloc": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp]),
             "psa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "psa_selftest_wait_timeout": (ctypes.c_int, [P, vp, sz, ctypes.c_uint64, vp]),
+            "psa_forward_host": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                ctypes.c_int, vp, vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -71,7 +73,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
             "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string",
-            "psa_forward_noalloc", "psa_selftest_wait_timeout")
+            "psa_forward_noalloc", "psa_selftest_wait_timeout", "psa_forward_host")
 
 
 def status_string(status: int) -> str:
@@ -148,6 +150,29 @@ def forward(p: Params, Q, K, V, O, ws, lse=None, level_map=None, stream=None):
     _check(lib().psa_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
                              _ptr(level_map), _ptr(ws), ws.numel(), _stream(stream)),
            "psa_forward")
+
+
+def host_groups(p: Params) -> int:
+    """A head-group count for forward_host: up to 8 groups of whole GQA groups,
+    or the KV heads' query heads split evenly when there are fewer KV heads."""
+    if p.Hkv >= 8:
+        return 8
+    grp = p.Hq // p.Hkv
+    per = max(1, min(grp, 8 // p.Hkv))
+    return p.Hkv * per
+
+
+def forward_host(p: Params, hQ, hK, hV, hO, Q, K, V, O, ws, h2d_stream, d2h_stream,
+                 hlse=None, lse=None, groups: Optional[int] = None, stream=None):
+    """psa_forward_host: the forward pass from (pinned) host tensors hQ, hK,
+    hV into hO (and hlse), with per-head-group copies on the two copy streams
+    pipelined behind the kernels on `stream`.  Q, K, V, O (and lse): device
+    buffers for the whole problem."""
+    g = host_groups(p) if groups is None else groups
+    _check(lib().psa_forward_host(ctypes.byref(p), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO),
+                                  _ptr(hlse), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                  _ptr(ws), ws.numel(), int(g), _stream(stream),
+                                  _stream(h2d_stream), _stream(d2h_stream)), "psa_forward_host")
 
 
 def forward_noalloc(p: Params, Q, K, V, O, lse=None, level_map=None, stream=None):

@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = ["pyramid.cu", "mask.cu", "score_tc.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu",
-           "psa_noalloc.cu", "psa_selftest.cu"]
+           "psa_noalloc.cu", "psa_selftest.cu", "psa_host.cu"]
 LIB = os.path.join(HERE, "libpsa.so")
 
 

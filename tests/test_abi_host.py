@@ -101,6 +101,23 @@ def test_assign_rule_validated():
     assert P.workspace_size(p) == 0                                   # unknown rule
 
 
+def test_forward_host_argument_errors_before_any_launch():
+    p = P.make_params(1, 4, 2, 1024, 64)
+    need = P.workspace_size(p)
+    A, B = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    S1, S2, S3 = ctypes.c_void_p(0x1), ctypes.c_void_p(0x2), ctypes.c_void_p(0x3)
+    f = lambda ws, groups, s1, s2, s3, hq=A: P.lib().psa_forward_host(
+        ctypes.byref(p), hq, A, A, A, None, A, A, A, A, None, ws, need, groups, s1, s2, s3)
+    assert f(B, 2, S1, S2, S2) == 1                                 # copy streams not distinct
+    assert f(B, 2, S1, S1, S3) == 1
+    assert f(B, 2, S1, S2, S3, hq=None) == 1                        # NULL host buffer
+    assert f(B, 0, S1, S2, S3) == 1                                 # no groups
+    assert f(B, 3, S1, S2, S3) == 1                                 # 3 groups cannot split 2 KV heads
+    assert f(B, 8, S1, S2, S3) == 1                                 # more groups than query heads
+    assert P.lib().psa_forward_host(ctypes.byref(p), A, A, A, A, None, A, A, A, A, None, B,
+                                    need - 1, 2, S1, S2, S3) == 4   # workspace too small
+
+
 def test_status_strings():
     for s in range(7):
         assert P.status_string(s)
