@@ -199,6 +199,44 @@ psa_status_t psa_forward_host(const psa_params_t* params, const void* Q_host, co
                               void* workspace, size_t workspace_bytes, int head_groups,
                               void* stream, void* h2d_stream, void* d2h_stream);
 
+/* Bytes of the scratch psa_backward needs besides the forward workspace (the
+ * per-row D = dO . O and the fp32 gradients of every pyramid level), or 0 if
+ * params is invalid. */
+size_t psa_backward_workspace_size(const psa_params_t* params);
+
+/* Gradient of the pyramid attention with the level map held fixed: dQ, dK,
+ * dV of the forward pass's O with respect to Q, K and V, given dO.
+ * Source: adaptive pyramid attention (top168.com article on PSA, component
+ * three) differentiated by the chain rule.  The map is a discrete function of
+ * Q and K and passes no gradient; the ln c logit bias is a constant.  With
+ * P_ig = exp(s q_i . K_l[g] + ln c_g - lse_i) over row i's kept keys,
+ * D_i = dO_i . O_i and dX_ig = P_ig (dO_i . V_l[g] - D_i):
+ *   dQ_i = s sum_g dX_ig K_l[g],
+ *   dK_l[g] = s sum_i dX_ig q_i,  dV_l[g] = sum_i P_ig dO_i,
+ * and each pooled row's gradient, divided by its token count c_g, goes to
+ * each of the c_g tokens it averages.  A KV head's gradients sum over the
+ * query heads that read it.  Rows that kept no key pass no gradient.
+ *  Q, K, V, O, dO: device, layouts of psa_forward; O and lse are the forward
+ *    pass's outputs for the same inputs and map.
+ *  lse: device fp32 [B, Hq, N], natural log, required.
+ *  level_map: device int8 [B, Hq, Nq, Nk] or NULL.  NULL: the work list the
+ *    last forward call left in `workspace` is used (so call this after
+ *    psa_forward / psa_attention_fwd with the same workspace); else the list
+ *    is rebuilt from the map, as psa_attention_fwd does.
+ *  workspace: the forward workspace, psa_workspace_size(params) bytes; the
+ *    pyramid levels in it are rebuilt from K and V.
+ *  bwd_workspace: device, 256-byte aligned, psa_backward_workspace_size(params)
+ *    bytes; caller-owned scratch, overwritten.
+ *  dQ [B, Hq, N, d], dK, dV [B, Hkv, N, d]: device outputs in the input dtype,
+ *    16-byte aligned; every element is written.
+ * Asynchronous on `stream`.  Errors as psa_forward (PSA_ERR_INVALID_ARG for a
+ * NULL lse or bwd_workspace). */
+psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void* K, const void* V,
+                          const void* O, const float* lse, const void* dO,
+                          const int8_t* level_map, void* workspace, size_t workspace_bytes,
+                          void* bwd_workspace, size_t bwd_workspace_bytes, void* dQ, void* dK,
+                          void* dV, void* stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
  * check, PSA_ERR_CUDA if the stream reported an error, else PSA_OK. */

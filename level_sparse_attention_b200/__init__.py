@@ -63,6 +63,9 @@ def lib() -> ctypes.CDLL:
             "psa_selftest_wait_timeout": (ctypes.c_int, [P, vp, sz, ctypes.c_uint64, vp]),
             "psa_forward_host": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                 ctypes.c_int, vp, vp, vp]),
+            "psa_backward_workspace_size": (sz, [P]),
+            "psa_backward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp, vp,
+                                            vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -73,7 +76,8 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
             "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string",
-            "psa_forward_noalloc", "psa_selftest_wait_timeout", "psa_forward_host")
+            "psa_forward_noalloc", "psa_selftest_wait_timeout", "psa_forward_host",
+            "psa_backward_workspace_size", "psa_backward")
 
 
 def status_string(status: int) -> str:
@@ -173,6 +177,27 @@ def forward_host(p: Params, hQ, hK, hV, hO, Q, K, V, O, ws, h2d_stream, d2h_stre
                                   _ptr(hlse), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
                                   _ptr(ws), ws.numel(), int(g), _stream(stream),
                                   _stream(h2d_stream), _stream(d2h_stream)), "psa_forward_host")
+
+
+def backward_workspace_size(p: Params) -> int:
+    return int(lib().psa_backward_workspace_size(ctypes.byref(p)))
+
+
+def new_backward_workspace(p: Params, device="cuda") -> torch.Tensor:
+    n = backward_workspace_size(p)
+    if n == 0:
+        raise PSAError(1, "psa_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def backward(p: Params, Q, K, V, O, lse, dO, ws, bws, dQ, dK, dV, level_map=None, stream=None):
+    """psa_backward: dQ, dK, dV of the pyramid attention with the map held
+    fixed.  ``ws`` is the forward workspace (its work list is used unless
+    ``level_map`` is given); ``bws`` the backward scratch."""
+    _check(lib().psa_backward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                              _ptr(dO), _ptr(level_map), _ptr(ws), ws.numel(), _ptr(bws),
+                              bws.numel(), _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream)),
+           "psa_backward")
 
 
 def forward_noalloc(p: Params, Q, K, V, O, lse=None, level_map=None, stream=None):

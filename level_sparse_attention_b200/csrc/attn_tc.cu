@@ -41,15 +41,17 @@
 #include <cudaTypedefs.h>
 
 #include "sm100_ptx.cuh"
+#include "tile_walk.cuh"
 #include "tma_host.cuh"
 
 namespace psa {
 namespace {
 
 using namespace ptx;
+using namespace tile;
 
 constexpr int kBM = 128;                 // query rows per CTA
-constexpr int kBN = 128;                 // keys per packed tile
+constexpr int kBN = kTileKeys;           // keys per packed tile
 constexpr int kStreams = 2;              // softmax warpgroups, one per stream of tiles
 constexpr int kVWarp = 2;                // the V producer
 constexpr int kSoftWarp0 = 4;            // first softmax warp (warpgroup aligned)
@@ -57,7 +59,6 @@ constexpr int kThreads = 128 + 128 * kStreams;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
-constexpr int kListCache = 1024;         // work-list entries staged in shared memory
 
 template <int D>
 struct Cfg {
@@ -148,60 +149,6 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 // How many of every 8 exponential pairs of a softmax tile take the FMA-pipe
 // polynomial above, the rest the transcendental unit (MUFU).
 constexpr int kPolyPairs = 0;
-
-// ------------------------------------------------------------ work list
-
-// Per query block: entry counts per level give where each level starts in
-// the entry list (f1..f4) and in the packed key sequence (b1..b4).  Kept in
-// scalars (no arrays) so that lookups by a run-time level stay in registers.
-struct RowWork {
-  int f1, f2, f3, f4;       // first entry of level 1, 2, 3; number of entries
-  int b1, b2, b3, b4;       // first packed key of level 1, 2, 3; number of keys
-  int tiles;
-};
-
-__device__ __forceinline__ RowWork row_work(int4 c) {
-  RowWork w;
-  w.f1 = c.x;
-  w.f2 = w.f1 + c.y;
-  w.f3 = w.f2 + c.z;
-  w.f4 = w.f3 + c.w;
-  w.b1 = 64 * c.x;
-  w.b2 = w.b1 + 32 * c.y;
-  w.b3 = w.b2 + 16 * c.z;
-  w.b4 = w.b3 + 8 * c.w;
-  w.tiles = (w.b4 + kBN - 1) / kBN;
-  return w;
-}
-
-__device__ __forceinline__ int sel4(int l, int a0, int a1, int a2, int a3) {
-  return l == 0 ? a0 : (l == 1 ? a1 : (l == 2 ? a2 : a3));
-}
-
-// The entries of tile t, one per lane: lane i takes the tile's first entry + i.
-// Entries never cross a tile edge, so the lanes inside the tile form a prefix.
-struct TileEntry {
-  bool in_tile;
-  int j, l, R, r0;          // KV block, level, sub-block rows, first row in the tile
-};
-
-__device__ __forceinline__ TileEntry tile_entry(const RowWork& w, const int* lrow,
-                                                const int* lcache, int t, int lane) {
-  // first entry of tile t: packed offset 128*t is always an entry boundary
-  const int off0 = t * kBN;
-  const int l0 = (off0 >= w.b1) + (off0 >= w.b2) + (off0 >= w.b3);
-  const int e = sel4(l0, 0, w.f1, w.f2, w.f3) + ((off0 - sel4(l0, 0, w.b1, w.b2, w.b3)) >> (6 - l0)) +
-                lane;
-  TileEntry te;
-  const int l = (e >= w.f1) + (e >= w.f2) + (e >= w.f3);
-  te.l = l;
-  te.R = 64 >> l;
-  const int off = sel4(l, 0, w.b1, w.b2, w.b3) + ((e - sel4(l, 0, w.f1, w.f2, w.f3)) << (6 - l));
-  te.in_tile = e < w.f4 && off < (t + 1) * kBN;
-  te.r0 = off - t * kBN;
-  te.j = te.in_tile ? (e < kListCache ? lcache[e] : __ldg(lrow + e)) : 0;
-  return te;
-}
 
 // Items (query blocks) of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
 // Consecutive CTAs take consecutive query blocks of the same head, so the

@@ -3,6 +3,7 @@
 #include <math.h>
 #include <string.h>
 
+#include "bwd_internal.cuh"
 #include "psa_internal.cuh"
 
 namespace psa {
@@ -146,6 +147,43 @@ psa_status_t psa_forward(const psa_params_t* params, const void* Q, const void* 
   if ((r = run_pyramid(params, L, K, V, workspace, st)) != PSA_OK) return r;
   if ((r = run_mask(params, L, Q, workspace, level_map, nullptr, st)) != PSA_OK) return r;
   return run_attention(params, L, Q, K, V, workspace, nullptr, O, lse, st);
+}
+
+size_t psa_backward_workspace_size(const psa_params_t* params) {
+  if (validate(params) != PSA_OK) return 0;
+  return make_bwd_layout(*params).total;
+}
+
+psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void* K, const void* V,
+                          const void* O, const float* lse, const void* dO,
+                          const int8_t* level_map, void* workspace, size_t workspace_bytes,
+                          void* bwd_workspace, size_t bwd_workspace_bytes, void* dQ, void* dK,
+                          void* dV, void* stream) {
+  psa_status_t r = validate(params);
+  if (r != PSA_OK) return r;
+  Layout L;
+  if ((r = check_ws(params, workspace, workspace_bytes, &L)) != PSA_OK) return r;
+  if ((r = check_ptrs({Q, K, V, O, dO, dQ, dK, dV})) != PSA_OK) return r;
+  if (!lse || !bwd_workspace) return PSA_ERR_INVALID_ARG;
+  if (!aligned4(lse) || (reinterpret_cast<uintptr_t>(bwd_workspace) & 255u) != 0)
+    return PSA_ERR_MISALIGNED;
+  const BwdLayout B = make_bwd_layout(*params);
+  if (bwd_workspace_bytes < B.total) return PSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = (cudaStream_t)stream;
+  BwdArgs a;
+  a.Q = Q; a.K = K; a.V = V; a.O = O; a.dO = dO; a.lse = lse;
+  a.dQ = dQ; a.dK = dK; a.dV = dV;
+  a.ws = (char*)workspace;
+  a.bws = (char*)bwd_workspace;
+  a.scale = scale_of(params);
+  if ((r = run_pyramid(params, L, K, V, workspace, st)) != PSA_OK) return r;
+  if (level_map && (r = from_cuda(launch_map_to_list(*params, L, level_map, (char*)workspace, st))) != PSA_OK)
+    return r;
+  if ((r = from_cuda(launch_bwd_prep(*params, B, a, st))) != PSA_OK) return r;
+  r = from_cuda(attention_bwd_tc_supported(*params) ? launch_attention_bwd_tc(*params, L, B, a, st)
+                                                    : launch_attention_bwd_simt(*params, L, B, a, st));
+  if (r != PSA_OK) return r;
+  return from_cuda(launch_bwd_unpool(*params, B, a, st));
 }
 
 psa_status_t psa_check_device(const psa_params_t* params, void* workspace, size_t workspace_bytes,

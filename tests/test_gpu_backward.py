@@ -1,0 +1,166 @@
+"""GPU parity of psa_backward (dQ, dK, dV with the level map held fixed)
+against the float64 backward oracle, through the C ABI.
+
+Tolerance (bf16 path), per gradient tensor, relative to its largest reference
+magnitude: max |err| <= 3e-2 and mean |err| / mean |ref| <= 1e-2.  The kernel
+stores P and dS = P (dP - D) in bf16 for the tensor-core products (relative
+rounding 2^-9 ~ 2e-3 each), reads the bf16-stored pyramid levels and the
+bf16 forward output O (through D = dO . O), and rounds the gradients to bf16
+once; the fp32 accumulation over many keys and query rows averages those
+roundings.  The fp32 CUDA-core path: max |err| <= 1e-4 of the largest
+magnitude."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import level_sparse_attention_b200 as P
+import oracle as O
+import workloads as W
+from oracle import psa_backward as OB
+from tests import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+BASE = W.BY_NAME
+CASES = {
+    # tensor-core path, d = 128, ragged N = 1000
+    "bf16_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, grid=(1, 20, 50),
+                                  coarse=(1, 5, 13), seed=41, target="fixed"),
+    # tensor-core path, d = 64, N = 226 + 760 with a forced text prefix
+    "bf16_d64": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, grid=(1, 20, 38),
+                                 coarse=(1, 5, 10), seed=42, target="fixed"),
+    # grouped queries (2 per KV head), causal
+    "bf16_gqa_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=4, Hkv=2, grid=(1, 25, 40),
+                                        coarse=(1, 7, 10), seed=43, target="fixed"),
+    # ragged pooled groups: N = 1003 (the last level-3 group averages 3 tokens)
+    "bf16_ragged_groups": W.with_overrides(BASE["wan2.1_1.3b"], Hq=1, Hkv=1, grid=(1, 17, 59),
+                                           coarse=(1, 5, 15), seed=44, target="fixed"),
+    # two batch elements
+    "bf16_batch2": W.with_overrides(BASE["wan2.1_1.3b"], B=2, Hq=1, Hkv=1, grid=(1, 16, 40),
+                                    coarse=(1, 4, 10), seed=45, target="fixed"),
+    # CUDA-core path: bf16 with 64-row query blocks, causal, grouped queries
+    "bf16_q64_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 20, 33),
+                                        coarse=(1, 5, 9), seed=46, q_blk=64, target="fixed"),
+    # CUDA-core path: fp32, d = 128 and the tiny fp32 workload (d = 64)
+    "f32_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, dtype="f32",
+                                 grid=(1, 18, 40), coarse=(1, 5, 10), seed=47, target="fixed"),
+    "tiny_f32": BASE["tiny_f32"],
+}
+
+
+def _map(w, kind, rng):
+    m = np.empty((w.B, w.Hq, w.Nq, w.Nk), dtype=np.int8)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            if kind == "random":
+                m[b, h] = G.rand_map(rng, w.Nq, w.Nk)
+            elif kind == "all_level0":
+                m[b, h] = 0
+            elif kind == "all_level3":
+                m[b, h] = 3
+            else:                                   # "pruned_rows"
+                m[b, h] = G.rand_map(rng, w.Nq, w.Nk, 0, 4)
+                m[b, h, 1::3] = -1
+            if w.causal:
+                for a in range(w.Nq):
+                    O.apply_overrides(m[b, h, a], a, w.N, w.q_blk, w.kv_blk, True, 0)
+                if kind == "pruned_rows":
+                    m[b, h, 1::3] = -1
+    return m
+
+
+def _grad_out(w, seed):
+    g = np.random.default_rng(seed).standard_normal((w.B, w.Hq, w.N, w.d)).astype(np.float32)
+    if w.dtype == "bf16":
+        bits = W.f32_to_bf16_bits(g)
+        return G.to_device(bits, "bf16"), W.bf16_bits_to_f32(bits).astype(np.float64)
+    return G.to_device(g, "f32"), g.astype(np.float64)
+
+
+def _run_backward(w, inp, run, dO, m=None):
+    p = run.p
+    dQ = torch.full_like(run.q, float("nan"))
+    dK = torch.full_like(run.k, float("nan"))
+    dV = torch.full_like(run.v, float("nan"))
+    bws = P.new_backward_workspace(p)
+    lm = None if m is None else torch.from_numpy(np.ascontiguousarray(m)).cuda()
+    P.backward(p, run.q, run.k, run.v, run.O, run.lse, dO, run.ws, bws, dQ, dK, dV, lm)
+    torch.cuda.synchronize()
+    P.check_device(p, run.ws)
+    return G.to_f64(dQ), G.to_f64(dK), G.to_f64(dV)
+
+
+def _oracle(w, inp, m, dO64):
+    Q, K, V = (np.stack([np.stack([inp.as_f64(n, b, h) for h in range(H)]) for b in range(w.B)])
+               for n, H in (("q", w.Hq), ("k", w.Hkv), ("v", w.Hkv)))
+    return OB.psa_backward(Q, K, V, dO64, m, w.q_blk, w.kv_blk, w.causal)
+
+
+def compare_grad(got, ref, dtype, what):
+    scale = max(float(np.abs(ref).max()), 1e-30)
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), what
+    max_rel = float(err.max()) / scale
+    mean_rel = float(err.mean() / max(np.abs(ref).mean(), 1e-30))
+    if dtype == "bf16":
+        assert max_rel <= 3e-2 and mean_rel <= 1e-2, (what, max_rel, mean_rel)
+    else:
+        assert max_rel <= 1e-4, (what, max_rel, mean_rel)
+    return max_rel, mean_rel
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("kind", ["random", "all_level0", "all_level3", "pruned_rows"])
+def test_backward_on_external_maps(name, kind):
+    w = CASES[name]
+    inp = W.make_inputs(w)
+    rng = np.random.default_rng(zlib.crc32(f"bwd/{name}/{kind}".encode()))
+    m = _map(w, kind, rng)
+    run = G.run_stages(w, inp, external_map=m)
+    dO, dO64 = _grad_out(w, zlib.crc32(f"dO/{name}".encode()))
+    gq, gk, gv = _run_backward(w, inp, run, dO, m)
+    ref = _oracle(w, inp, m, dO64)
+    compare_grad(gq, ref.dQ, w.dtype, "dQ")
+    compare_grad(gk, ref.dK, w.dtype, "dK")
+    compare_grad(gv, ref.dV, w.dtype, "dV")
+    if kind == "pruned_rows":
+        # query blocks that keep nothing pass no gradient: dQ rows exactly 0
+        for a in range(1, w.Nq, 3):
+            rows = slice(a * w.q_blk, min((a + 1) * w.q_blk, w.N))
+            assert np.all(gq[:, :, rows] == 0)
+
+
+@pytest.mark.parametrize("name", ["bf16_d128", "bf16_gqa_causal", "tiny_f32"])
+def test_backward_after_fused_forward_uses_its_work_list(name):
+    """level_map = NULL: the backward walks the list psa_forward left in the
+    workspace; the oracle is given the map the GPU chose."""
+    w = CASES[name]
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp, fused=True)
+    gm = run.level_map.cpu().numpy()
+    dO, dO64 = _grad_out(w, 99)
+    gq, gk, gv = _run_backward(w, inp, run, dO, None)
+    ref = _oracle(w, inp, gm, dO64)
+    compare_grad(gq, ref.dQ, w.dtype, "dQ")
+    compare_grad(gk, ref.dK, w.dtype, "dK")
+    compare_grad(gv, ref.dV, w.dtype, "dV")
+
+
+def test_backward_invariants_on_gpu():
+    """Properties that hold at any size, on the tensor-core path: the dV sum
+    equals the dO sum over rows that keep a key, and dK sums to 0."""
+    w = CASES["bf16_d128"]
+    inp = W.make_inputs(w)
+    m = _map(w, "random", np.random.default_rng(5))
+    run = G.run_stages(w, inp, external_map=m)
+    dO, dO64 = _grad_out(w, 7)
+    gq, gk, gv = _run_backward(w, inp, run, dO, m)
+    live = np.isfinite(run.lse.cpu().numpy())
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            want = (dO64[b, h] * live[b, h][:, None]).sum(0)
+            scale = np.abs(dO64[b, h]).sum(0).max()
+            assert np.abs(gv[b, h].sum(0) - want).max() <= 1e-2 * scale
+            assert np.abs(gk[b, h].sum(0)).max() <= 1e-2 * np.abs(gk[b, h]).sum(0).max()
