@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-heads", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward-pass measurement")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: run only this many query heads (KV heads scaled to match)")
     ap.add_argument("--profile-kernels", action="store_true",
@@ -60,14 +62,18 @@ def parse():
 # its query heads and a hash of the attention kernel's sources.  A kernel that
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
-ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "27cc7203d4316d64"): 473.676032e6 + 93.238528e6}
+ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
+ATTN_TRAFFIC = {}
+# the same for one launch of the attention-gradient kernel
+BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
+               "bwd_internal.cuh")
+BWD_TRAFFIC = {}
 
 
-def attn_source_hash() -> str:
+def attn_source_hash(sources=ATTN_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ATTN_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, "level_sparse_attention_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -361,6 +367,46 @@ def run_ours(args, rank, world, local_rank):
     job_dense = dense * world if args.shard == "batch" else w_job.dense_flops()
     P.check_device(p, ws)
 
+    # the backward pass (dQ, dK, dV with this map held fixed), timed the same
+    # way: L2 flushed between steps, CUDA events on the launch stream.  Its
+    # executed FLOPs are 5 tile GEMMs (S, dP, dQ, dK, dV) against the
+    # forward's 2, over the same packed tiles.
+    bwd = None
+    if not args.no_backward:
+        gen = torch.Generator(device=dev).manual_seed(1234)
+        dout = torch.randn(out.shape, generator=gen, device=dev, dtype=torch.float32).to(out.dtype)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = P.new_backward_workspace(p, dev)
+
+        def bstep():
+            P.backward(p, q, k, v, out, lse, dout, ws, bws, dq, dk, dv)
+
+        step()                                   # the forward this backward belongs to
+        for _ in range(max(3, args.warmup)):
+            bstep()
+        torch.cuda.synchronize()
+        P.check_device(p, ws)
+        b_steps = max(3, min(args.steps, 20))
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(b_steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(b_steps):
+            flush.zero_()
+            bev[i][0].record(stream)
+            bstep()
+            bev[i][1].record(stream)
+        torch.cuda.synchronize()
+        P.check_device(p, ws)
+        b_ms = max_over_ranks(sum(b[0].elapsed_time(b[1]) for b in bev) / b_steps, world, dev)
+        b_exec = 2.5 * executed
+        bwd = {"ms_per_call": b_ms, "steps": b_steps, "call": "psa_backward",
+               "stages": "pyramid rebuild, D = dO . O, attention gradient, unpool",
+               "executed_flops": b_exec,
+               "executed_tflops": b_exec * (world if args.shard == "batch" else 1) / (b_ms * 1e-3) / 1e12,
+               "dense_equiv_tflops": 2.5 * (job_dense / (b_ms * 1e-3) / 1e12),
+               "traffic": BWD_TRAFFIC.get((w.name, w.Hq, attn_source_hash(BWD_SOURCES))),
+               "gpu_launches_per_call": 4}
     kernels_us = None
     if args.profile_kernels:
         # per-kernel device times over extra steps (not the timed ones)
@@ -369,6 +415,9 @@ def run_ours(args, rank, world, local_rank):
             for _ in range(args.steps):
                 flush.zero_()
                 step()
+                if bwd is not None:
+                    flush.zero_()
+                    bstep()
             torch.cuda.synchronize()
         agg = {}
         for e in prof.events():
@@ -386,6 +435,9 @@ def run_ours(args, rank, world, local_rank):
     mask_avg = sum(mask_ms) / len(mask_ms)
     pyr_gbs = pyramid_bytes(w) / (pyr_avg * 1e-3) / 1e9
     mask_gbs = mask_bytes(w) / (mask_avg * 1e-3) / 1e9
+    if bwd is not None:
+        bwd["frac_of_peak"] = bwd["executed_tflops"] / (world if args.shard == "batch" else 1) / bf16_peak
+        bwd["peak_kind"] = f"{peak_kind} bf16 burst"
     if rank != 0:
         return
     cpu, parity = None, None
@@ -419,6 +471,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": ATTN_TRAFFIC.get((w.name, w.Hq, attn_source_hash())),
                      "executed_flops_per_launch": executed,
                      "padding_fraction": 1.0 - (keys_per_row.sum() / max(padded_keys, 1.0))},
+        "backward": bwd,
         "cpu_baseline": cpu,
         "parity": parity,
         "e2e": {"value": job_dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,

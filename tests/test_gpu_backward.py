@@ -71,15 +71,20 @@ def _map(w, kind, rng):
     return m
 
 
-def _grad_out(w, seed):
+def _grad_out(w, seed, wide=True):
+    """dO: seeded N(0, 1) in the workload's dtype, on the device, and the same
+    values on the host (float64 if ``wide``, else float32)."""
     g = np.random.default_rng(seed).standard_normal((w.B, w.Hq, w.N, w.d)).astype(np.float32)
     if w.dtype == "bf16":
         bits = W.f32_to_bf16_bits(g)
-        return G.to_device(bits, "bf16"), W.bf16_bits_to_f32(bits).astype(np.float64)
-    return G.to_device(g, "f32"), g.astype(np.float64)
+        g = W.bf16_bits_to_f32(bits)
+        dev = G.to_device(bits, "bf16")
+    else:
+        dev = G.to_device(g, "f32")
+    return dev, (g.astype(np.float64) if wide else g)
 
 
-def _run_backward(w, inp, run, dO, m=None):
+def _run_backward(w, inp, run, dO, m=None, host=True):
     p = run.p
     dQ = torch.full_like(run.q, float("nan"))
     dK = torch.full_like(run.k, float("nan"))
@@ -89,6 +94,9 @@ def _run_backward(w, inp, run, dO, m=None):
     P.backward(p, run.q, run.k, run.v, run.O, run.lse, dO, run.ws, bws, dQ, dK, dV, lm)
     torch.cuda.synchronize()
     P.check_device(p, run.ws)
+    del bws
+    if not host:
+        return dQ, dK, dV
     return G.to_f64(dQ), G.to_f64(dK), G.to_f64(dV)
 
 
@@ -164,3 +172,69 @@ def test_backward_invariants_on_gpu():
             scale = np.abs(dO64[b, h]).sum(0).max()
             assert np.abs(gv[b, h].sum(0) - want).max() <= 1e-2 * scale
             assert np.abs(gk[b, h].sum(0)).max() <= 1e-2 * np.abs(gk[b, h]).sum(0).max()
+
+
+FULL = ["wan2.1_1.3b", "cogvideox_5b", "wan2.1_14b_720p", "qwen2.5_vl_7b"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_backward_full_size_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration.
+    1. The map the GPU chose: dQ of sampled query blocks (each depends only on
+       its own kept keys) against the oracle, and the dK / dV sums that hold
+       at any size (sum dV = sum dO over rows that keep a key; sum dK = 0).
+    2. A map keeping only a few query blocks of a few heads: every element of
+       dQ, dK and dV against the oracle (only those blocks contribute)."""
+    w = W.BY_NAME[name]
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp, fused=True)
+    gm = run.level_map.cpu().numpy()
+    dO, dO32 = _grad_out(w, 2024, wide=False)
+    gq, gk, gv = _run_backward(w, inp, run, dO, None, host=False)
+    grp = w.Hq // w.Hkv
+    rng = np.random.default_rng(3)
+    heads = sorted({0, w.Hq // 2, w.Hq - 1})
+    blocks = sorted({0, w.Nq - 1, int(rng.integers(1, w.Nq - 1))})
+    s = 1.0 / np.sqrt(w.d)
+    for h in heads:
+        Q, dOh = inp.as_f64("q", 0, h), dO32[0, h].astype(np.float64)
+        K, V = inp.as_f64("k", 0, h // grp), inp.as_f64("v", 0, h // grp)
+        sub = np.full_like(gm[0, h], -1)
+        sub[blocks] = gm[0, h][blocks]
+        ref = OB.pyramid_attention_backward(Q, K, V, sub, dOh, w.q_blk, w.kv_blk, s, w.causal)
+        rows = np.concatenate([np.arange(a * w.q_blk, min((a + 1) * w.q_blk, w.N)) for a in blocks])
+        compare_grad(G.to_f64(gq[0, h])[rows], ref.dQ[rows], w.dtype, f"dQ head {h}")
+    live = torch.isfinite(run.lse[0]).to(torch.float64)                        # [Hq, N]
+    dO_dev = dO[0].to(torch.float64) * live[:, :, None]
+    for hk in range(w.Hkv):
+        want = dO_dev[hk * grp:(hk + 1) * grp].sum((0, 1))
+        v64, k64 = gv[0, hk].to(torch.float64), gk[0, hk].to(torch.float64)
+        assert float((v64.sum(0) - want).abs().max()) <= 1e-2 * float(v64.abs().sum(0).max()), hk
+        assert float(k64.sum(0).abs().max()) <= 1e-2 * float(k64.abs().sum(0).max()), hk
+    del gq, gk, gv, dO_dev
+
+    # 2. a few query blocks of a few heads, every gradient element
+    sub = np.full_like(gm, -1)
+    for h in heads:
+        sub[0, h, blocks] = gm[0, h, blocks]
+    del run
+    run2 = G.run_stages(w, inp, external_map=sub)
+    gq, gk, gv = _run_backward(w, inp, run2, dO, sub, host=False)
+    kv_heads = sorted({h // grp for h in heads})
+    for hk in kv_heads:
+        K, V = inp.as_f64("k", 0, hk), inp.as_f64("v", 0, hk)
+        dK = np.zeros((w.N, w.d))
+        dV = np.zeros((w.N, w.d))
+        for h in [h for h in heads if h // grp == hk]:
+            ref = OB.pyramid_attention_backward(inp.as_f64("q", 0, h), K, V, sub[0, h],
+                                                dO32[0, h].astype(np.float64), w.q_blk, w.kv_blk,
+                                                s, w.causal)
+            compare_grad(G.to_f64(gq[0, h]), ref.dQ, w.dtype, f"dQ head {h}")
+            dK += ref.dK
+            dV += ref.dV
+        compare_grad(G.to_f64(gk[0, hk]), dK, w.dtype, f"dK kv head {hk}")
+        compare_grad(G.to_f64(gv[0, hk]), dV, w.dtype, f"dV kv head {hk}")
+    others = [h for h in range(w.Hkv) if h not in kv_heads]
+    if others:
+        assert bool((gk[0, others] == 0).all()) and bool((gv[0, others] == 0).all())
