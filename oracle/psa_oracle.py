@@ -197,6 +197,47 @@ def level_of_rank(rank: np.ndarray, K: np.ndarray) -> np.ndarray:
     return out
 
 
+def block_max_levels(K: np.ndarray, bk: int, theta: float,
+                     pool: Sequence[int] = POOL) -> Tuple[np.ndarray, np.ndarray]:
+    """Cosine-similarity constraint on the pyramid ([news] ablations name a
+    cosine-similarity constraint and its gain; the pages do not define it).
+
+    Reading: every pooled row of level l >= 1 merges two rows of level l - 1,
+    the token ranges [2g f', (2g+1) f') and [(2g+1) f', (2g+2) f') with
+    f' = f_(l-1), cut at N.  The merge is similar when the cosine of the two
+    halves' mean keys is >= theta; a merge whose second half is empty, or one
+    of whose halves has a zero mean, passes.  KV block j may be represented at
+    level l when every merge at levels 1..l inside it is similar.
+    Returns (max_level [Nk] int: the largest such l, or 0; min_cos [Nk, L+1]:
+    the smallest cosine among block j's merges at each level, +inf where a
+    level has no merge, column 0 unused)."""
+    N, _ = K.shape
+    L = len(pool) - 1
+    Nk = cdiv(N, bk)
+    min_cos = np.full((Nk, L + 1), np.inf)
+    for j in range(Nk):
+        for l in range(1, L + 1):
+            half = pool[l - 1]
+            for start in range(j * bk, min((j + 1) * bk, N), pool[l]):
+                a_lo, a_hi = start, min(start + half, N)
+                b_lo, b_hi = a_hi, min(start + pool[l], N)
+                if b_hi <= b_lo:
+                    continue                       # no second half: nothing merged
+                a = K[a_lo:a_hi].mean(axis=0)
+                b = K[b_lo:b_hi].mean(axis=0)
+                na, nb = np.linalg.norm(a), np.linalg.norm(b)
+                c = 1.0 if na == 0 or nb == 0 else float(a @ b) / (na * nb)
+                min_cos[j, l] = min(min_cos[j, l], c)
+    max_level = np.zeros(Nk, dtype=np.int64)
+    for j in range(Nk):
+        for l in range(1, L + 1):
+            if min_cos[j, l] >= theta:
+                max_level[j] = l
+            else:
+                break
+    return max_level, min_cos
+
+
 def apply_overrides(row: np.ndarray, a: int, N: int, bq: int, bk: int, causal: bool,
                     forced_prefix_tokens: int) -> None:
     """In place: causal blocks after the query block are pruned and blocks
@@ -213,7 +254,8 @@ def apply_overrides(row: np.ndarray, a: int, N: int, bq: int, bk: int, causal: b
 
 def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
                   causal: bool = False, forced_prefix_tokens: int = 0,
-                  rule: str = "threshold") -> MaskResult:
+                  rule: str = "threshold",
+                  max_level: Optional[np.ndarray] = None) -> MaskResult:
     """Multi-level mask ([news] ablations: threshold-based assignment, compared
     there with a quantile-based one; [abs] lower levels to critical blocks,
     higher to less important).
@@ -223,6 +265,9 @@ def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
     Threshold rule: level = the smallest l with C_r < tau_l, else pruned.
     Quantile rule: level = the smallest l with r < K_l = ceil(tau_l * n_visible)
     (``quotas``), else pruned.  Then the overrides of ``apply_overrides``.
+    With ``max_level`` (``block_max_levels``), every kept level is then
+    lowered to at most its block's max_level (finer, never coarser; pruned
+    blocks stay pruned).
     Readings: the exclusive cumulative mass (so the top block always gets
     level 0), the quotas as cumulative fractions of the visible blocks rounded
     up, and the override order are this build's."""
@@ -243,6 +288,9 @@ def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
         else:
             level_map[a, order] = level_of_rank(np.arange(len(order)), quotas(len(order), tau))
         apply_overrides(level_map[a], a, N, bq, bk, causal, forced_prefix_tokens)
+        if max_level is not None:
+            kept = level_map[a] >= 0
+            level_map[a, kept] = np.minimum(level_map[a, kept], max_level[kept])
     return MaskResult(level_map, mass, cum, rank)
 
 
@@ -309,15 +357,18 @@ class HeadResult:
 def psa_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, bq: int, bk: int,
              tau: Sequence[float], causal: bool = False, forced_prefix_tokens: int = 0,
              scale: Optional[float] = None, level_map: Optional[np.ndarray] = None,
-             pool: Sequence[int] = POOL, rule: str = "threshold") -> HeadResult:
+             pool: Sequence[int] = POOL, rule: str = "threshold",
+             sim_threshold: Optional[float] = None) -> HeadResult:
     """The whole PSA forward for one (batch, query head): pyramid, query-block
-    means, block logits, level assignment (unless ``level_map`` is given), then
+    means, block logits, level assignment (unless ``level_map`` is given; with
+    the cosine-similarity constraint when ``sim_threshold`` is given), then
     pyramid attention.  Q [N, d]; K, V [N, d] of the matching KV head."""
     N, d = Q.shape
     s = 1.0 / math.sqrt(d) if scale is None else scale
     pyr = build_pyramid(K, V, pool)
     z = block_logits(query_block_means(Q, bq), pyr, bk, s, pool)
-    mask = assign_levels(z, tau, N, bq, bk, causal, forced_prefix_tokens, rule)
+    ml = None if sim_threshold is None else block_max_levels(K, bk, sim_threshold, pool)[0]
+    mask = assign_levels(z, tau, N, bq, bk, causal, forced_prefix_tokens, rule, ml)
     lm = mask.level_map if level_map is None else level_map
     O, lse = pyramid_attention(Q, pyr, lm, bq, bk, s, causal, pool)
     return HeadResult(O, lse, mask, z)

@@ -356,4 +356,81 @@ def pin_attention_scale_shift(O):
     assert np.allclose(out, out2, atol=1e-13)
 
 
+# --------------------------------------------- cosine-similarity constraint
+
+def _rot(x, ang):
+    c, s_ = math.cos(ang), math.sin(ang)
+    return np.array([c * x[0] - s_ * x[1], s_ * x[0] + c * x[1]])
+
+
+def pin_similarity_closed_form_angles(O):
+    """Every 8-token group: tokens (u, u, v, v, R u, R u, R v, R v) with
+    angle(u, v) = 60 degrees and R a 30-degree rotation.  Level-1 merges join
+    equal tokens (cos 1), level-2 merges join u and v (cos 1/2), level-3 merges
+    join mean(u, v) and its rotation (cos 30 degrees)."""
+    u = np.array([1.0, 0.0])
+    v = _rot(u, math.pi / 3)
+    grp = [u, u, v, v, _rot(u, math.pi / 6), _rot(u, math.pi / 6), _rot(v, math.pi / 6),
+           _rot(v, math.pi / 6)]
+    K = np.array(grp * 16)                               # N = 128: two blocks of 64
+    ml, mc = O.block_max_levels(K, 64, 0.6)
+    assert np.allclose(mc[:, 1], 1.0) and np.allclose(mc[:, 2], 0.5)
+    assert np.allclose(mc[:, 3], math.cos(math.pi / 6))
+    assert list(ml) == [1, 1]                            # level 2 fails at 0.6, so level 3 is out
+    assert list(O.block_max_levels(K, 64, 0.4)[0]) == [3, 3]
+    assert list(O.block_max_levels(K, 64, 0.9)[0]) == [1, 1]
+    assert list(O.block_max_levels(K, 64, 1.0 + 1e-9)[0]) == [0, 0]
+
+
+def pin_similarity_orthogonal_opposite_ragged_zero(O):
+    """Exact cosines 0 and -1, an absent second half at the ragged end, and a
+    zero-mean half (which always passes)."""
+    e1, e2 = np.array([1.0, 0.0]), np.array([0.0, 1.0])
+    K = np.tile(e1, (64 + 3, 1))
+    K[1] = e2                                            # block 0: one orthogonal token pair
+    assert O.block_max_levels(K, 64, 0.0)[0][0] >= 1     # cos 0 >= 0 passes
+    assert O.block_max_levels(K, 64, 1e-6)[0][0] == 0
+    K = np.tile(e1, (64 + 3, 1))
+    K[66] = -e1                                          # block 1 = tokens 64, 65, 66
+    ml, mc = O.block_max_levels(K, 64, -0.5)
+    assert mc[1, 1] == 1.0                               # (64, 65); 66 has no partner
+    assert mc[1, 2] == -1.0                              # (64, 65) against (66)
+    assert np.isinf(mc[1, 3])                            # tokens 68.. do not exist
+    assert ml[1] == 1 and ml[0] == 3
+    K = np.tile(e1, (64, 1))
+    K[0] = 0.0                                           # zero-mean half: the merge passes
+    assert O.block_max_levels(K, 64, 0.99)[0][0] == 3
+
+
+def pin_similarity_scale_invariance(O):
+    """Cosines do not change when every key is scaled by a positive constant,
+    and every min cosine lies in [-1, 1]."""
+    rng = np.random.default_rng(17)
+    K = rng.standard_normal((200, 8)) + 2.0
+    a, ca = O.block_max_levels(K, 64, 0.8)
+    b, cb = O.block_max_levels(3.7 * K, 64, 0.8)
+    assert np.array_equal(a, b) and np.allclose(ca, cb)
+    fin = np.isfinite(ca[:, 1:])
+    assert np.all(np.abs(ca[:, 1:][fin]) <= 1 + 1e-12)
+
+
+def pin_similarity_clamps_assignment(O):
+    """The constraint only lowers kept levels (to min(level, max level)) and
+    never touches pruned blocks; theta = -1 changes nothing, and a theta no
+    random merge reaches leaves every kept block at level 0."""
+    rng = np.random.default_rng(19)
+    N, d, bq, bk = 64 * 9 + 5, 8, 64, 64
+    Q, K, V = rng.standard_normal((N, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    tau = (0.3, 0.5, 0.7, 0.9)
+    free = O.psa_head(Q, K, V, bq, bk, tau).mask.level_map
+    ml = rng.integers(0, 4, size=free.shape[1])
+    z = O.block_logits(O.query_block_means(Q, bq), O.build_pyramid(K, V), bk, 1 / math.sqrt(d))
+    got = O.assign_levels(z, tau, N, bq, bk, max_level=ml).level_map
+    want = np.where(free >= 0, np.minimum(free, ml[None, :]), -1)
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.psa_head(Q, K, V, bq, bk, tau, sim_threshold=-1.0).mask.level_map, free)
+    one = O.psa_head(Q, K, V, bq, bk, tau, sim_threshold=1.0).mask.level_map
+    assert np.array_equal(one, np.where(free >= 0, 0, -1))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

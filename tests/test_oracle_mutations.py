@@ -35,6 +35,15 @@ MUTATIONS = {
     "quantile tau in double": ("np.asarray(tau, dtype=np.float32).astype(np.float64)", "np.asarray(tau, dtype=np.float64)"),
     "quantile rank <= quota": ("out[rank < K[l]] = l", "out[rank <= K[l]] = l"),
     "quantile quotas of all blocks": ("quotas(len(order), tau)", "quotas(Nk, tau)"),
+    "similarity merge half shifted": ("b_lo, b_hi = a_hi, min(start + pool[l], N)",
+                                      "b_lo, b_hi = a_hi + 1, min(start + pool[l] + 1, N)"),
+    "similarity without normalisation": ("c = 1.0 if na == 0 or nb == 0 else float(a @ b) / (na * nb)",
+                                         "c = float(a @ b)"),
+    "similarity strict >": ("if min_cos[j, l] >= theta:", "if min_cos[j, l] > theta:"),
+    "similarity not cumulative": ("                max_level[j] = l\n            else:\n                break",
+                                  "                max_level[j] = l"),
+    "similarity clamp coarsens": ("np.minimum(level_map[a, kept], max_level[kept])",
+                                  "np.maximum(level_map[a, kept], max_level[kept])"),
 }
 
 
@@ -82,6 +91,8 @@ def test_mutation_is_caught_by_a_pin(name):
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught_by_bruteforce(name):
+    if name.startswith("similarity"):
+        pytest.skip("the constraint is off in the brute force's cases; its pins catch these")
     if name in ("threshold <= instead of <", "ties to the higher index", "quantile tau in double"):
         pytest.skip("random masses never tie or land on a threshold, and these quotas are exact "
                     "in both precisions; the golden cases pin these")
