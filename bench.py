@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass measurement")
+    ap.add_argument("--sim-threshold", type=float, default=-1.0,
+                    help="cosine-similarity constraint on the pyramid levels (-1: off, the "
+                         "method's default)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: run only this many query heads (KV heads scaled to match)")
     ap.add_argument("--profile-kernels", action="store_true",
@@ -137,7 +140,7 @@ def pyramid_bytes(w: W.Workload) -> float:
 
 # ------------------------------------------------------------- CPU oracle leg
 
-def cpu_sample(w: W.Workload, n_heads: int):
+def cpu_sample(w: W.Workload, n_heads: int, sim_threshold: float = -1.0):
     """Time the oracle (as it stands) on `n_heads` whole heads of the workload.
     Returns (dense-equivalent TFLOP/s, seconds, cores, sample description,
     the oracle's per-head results)."""
@@ -152,7 +155,8 @@ def cpu_sample(w: W.Workload, n_heads: int):
     for h in heads:
         results.append(O.psa_head(inp.as_f64("q", 0, h), inp.as_f64("k", 0, h // grp),
                                   inp.as_f64("v", 0, h // grp), w.q_blk, w.kv_blk, tau, w.causal,
-                                  w.forced_prefix_tokens))
+                                  w.forced_prefix_tokens,
+                                  sim_threshold=None if sim_threshold <= -1 else sim_threshold))
     dt = time.perf_counter() - t0
     dense = w.dense_flops() / (w.B * w.Hq) * n_heads
     return (dense / dt / 1e12, dt, cores,
@@ -283,7 +287,8 @@ def run_ours(args, rank, world, local_rank):
         inp = W.make_inputs(w, batch0=rank_batch0(rank, w.B))
     p = P.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.q_blk, w.kv_blk, tau, w.causal,
                       w.forced_prefix_tokens, 0.0,
-                      torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+                      torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                      sim_threshold=args.sim_threshold)
 
     def host(x):
         t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
@@ -442,7 +447,7 @@ def run_ours(args, rank, world, local_rank):
         return
     cpu, parity = None, None
     if not args.no_cpu_baseline and world == 1:
-        val, dt, cores, sample, results = cpu_sample(w, args.cpu_sample_heads)
+        val, dt, cores, sample, results = cpu_sample(w, args.cpu_sample_heads, args.sim_threshold)
         cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(dt, 2)}
         parity = sampled_parity(w, results, lm, out)
@@ -456,6 +461,7 @@ def run_ours(args, rank, world, local_rank):
                    "shard": args.shard, "B": w.B, "Hq": w_job.Hq, "Hkv": w_job.Hkv, "N": w.N, "d": w.d,
                    "q_blk": w.q_blk, "kv_blk": w.kv_blk, "tau": [round(t, 6) for t in tau],
                    "causal": w.causal, "skipped_dense_fraction": 1.0 - executed / dense,
+                   "sim_threshold": args.sim_threshold,
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": (f"independent batch per GPU x{world}" if args.shard == "batch"
                                    else f"heads of one problem split over {world} GPUs")},

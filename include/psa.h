@@ -79,7 +79,18 @@ typedef enum { PSA_ASSIGN_THRESHOLD = 0, PSA_ASSIGN_QUANTILE = 1 } psa_assign_t;
  *  assign            level assignment rule (psa_assign_t): threshold on the
  *                    cumulative mass (the method's rule) or per-level quotas of
  *                    blocks by rank (the quantile-based rule the method is
- *                    compared with: top168.com article on PSA, ablations).   */
+ *                    compared with: top168.com article on PSA, ablations).
+ *  sim_threshold     cosine-similarity constraint on the pyramid (the article's
+ *                    ablations name such a constraint without defining it; this
+ *                    is the library's reading).  Every pooled row of level
+ *                    l >= 1 merges two rows of level l - 1; a merge is similar
+ *                    when the cosine of its halves' mean keys is >=
+ *                    sim_threshold (an empty or zero half passes).  A KV block
+ *                    may use level l only when every merge at levels 1..l inside
+ *                    it is similar; kept levels above that are lowered to it
+ *                    (per KV head, after the overrides).  In [-1, 1]; -1 turns
+ *                    the constraint off (every cosine passes), and so does any
+ *                    value below -1.  NaN or a value above 1 is rejected.    */
 typedef struct {
   int B, Hq, Hkv, N, d;
   int q_blk, kv_blk;
@@ -91,13 +102,15 @@ typedef struct {
   float scale;
   psa_dtype_t dtype;
   psa_assign_t assign;
+  float sim_threshold;
 } psa_params_t;
 
 /* Bytes of device workspace the calls below need for `params` (0 if params are
  * invalid).  The workspace holds: a device error word; pooled K/V levels 1..3
  * [B, Hkv, ceil(N/2^l), d] in dtype; level-3 keys in fp32 for scoring;
- * query-block means; block logits; an internal level map; and the per-query-
- * block work list (KV block indices sorted by level, then index).  It is owned
+ * query-block means; block logits; an internal level map; the per-KV-block
+ * largest level the cosine constraint allows; and the per-query-block work
+ * list (KV block indices sorted by level, then index).  It is owned
  * by the caller and may be reused across calls with the same params. */
 size_t psa_workspace_size(const psa_params_t* params);
 
@@ -105,7 +118,9 @@ size_t psa_workspace_size(const psa_params_t* params);
  * component one: bottom level = original KV, each level up average-pooled).
  * K, V: device [B, Hkv, N, d].  Writes levels 1..3 of K and V and the fp32
  * level-3 keys into `workspace`.  Pooled row g of level l is the mean of tokens
- * [g*2^l, min((g+1)*2^l, N)), summed in fp32 and rounded once to dtype. */
+ * [g*2^l, min((g+1)*2^l, N)), summed in fp32 and rounded once to dtype.
+ * With sim_threshold > -1 it also records, per KV head and block, the largest
+ * level the cosine-similarity constraint allows (cosines in fp32). */
 psa_status_t psa_build_pyramid(const psa_params_t* params, const void* K, const void* V,
                                void* workspace, size_t workspace_bytes, void* stream);
 

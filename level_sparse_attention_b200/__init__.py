@@ -36,7 +36,8 @@ class Params(ctypes.Structure):
                 ("kv_blk", ctypes.c_int), ("n_levels", ctypes.c_int),
                 ("pool", ctypes.c_int * 4), ("tau", ctypes.c_float * 4),
                 ("causal", ctypes.c_int), ("forced_prefix_tokens", ctypes.c_int),
-                ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("assign", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("assign", ctypes.c_int),
+                ("sim_threshold", ctypes.c_float)]
 
 
 _lib = None
@@ -93,7 +94,10 @@ ASSIGN_THRESHOLD, ASSIGN_QUANTILE = 0, 1
 def make_params(B: int, Hq: int, Hkv: int, N: int, d: int, q_blk: int = 128, kv_blk: int = 64,
                 tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97), causal: bool = False,
                 forced_prefix_tokens: int = 0, scale: float = 0.0,
-                dtype: torch.dtype = torch.bfloat16, assign: int = ASSIGN_THRESHOLD) -> Params:
+                dtype: torch.dtype = torch.bfloat16, assign: int = ASSIGN_THRESHOLD,
+                sim_threshold: float = -1.0) -> Params:
+    """psa_params_t for the arguments; ``sim_threshold`` > -1 turns on the
+    cosine-similarity constraint on the pyramid levels."""
     p = Params()
     p.B, p.Hq, p.Hkv, p.N, p.d = B, Hq, Hkv, N, d
     p.q_blk, p.kv_blk, p.n_levels = q_blk, kv_blk, 4
@@ -103,6 +107,7 @@ def make_params(B: int, Hq: int, Hkv: int, N: int, d: int, q_blk: int = 128, kv_
     p.causal, p.forced_prefix_tokens, p.scale = int(bool(causal)), forced_prefix_tokens, scale
     p.dtype = BF16 if dtype == torch.bfloat16 else F32
     p.assign = int(assign)
+    p.sim_threshold = float(sim_threshold)
     return p
 
 
@@ -313,6 +318,7 @@ def workspace_layout(p: Params) -> dict:
     L["qml"], off = off, off + a256(rq * p.d * 4)
     L["zlog"], off = off, off + a256(rq * Nk * 4)
     L["map"], off = off, off + a256(rq * Nk)
+    L["maxlev"], off = off, off + a256(p.B * p.Hkv * Nk)
     L["counts"], off = off, off + a256(rq * 16)
     L["list"], off = off, off + a256(rq * Nk * 4)
     L["total"] = off

@@ -304,7 +304,8 @@ __device__ __forceinline__ void levels_from_sorted(const unsigned long long (&v)
 
 template <int K>
 __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
-                              const float* __restrict__ zlog, int8_t* __restrict__ map_ws,
+                              const float* __restrict__ zlog, const int8_t* __restrict__ maxlev,
+                              int8_t* __restrict__ map_ws,
                               int8_t* __restrict__ map_user, float* __restrict__ mass_user,
                               int* __restrict__ list, int4* __restrict__ counts) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -608,6 +609,16 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
     if (strad || forced) lev[j] = 0;
   }
   __syncwarp();
+  if (a.sim_threshold > -1.f) {
+    // cosine-similarity constraint: a kept block's level is lowered to the
+    // largest its KV head's merges allow (pruned blocks stay pruned)
+    const int bhq = row / a.Nq;
+    const int bhk = (bhq / a.Hq) * a.Hkv + (bhq % a.Hq) / (a.Hq / a.Hkv);
+    const int8_t* ml = maxlev + (long long)bhk * a.Nk;
+    for (int j = lane; j < a.Nk; j += 32)
+      if (lev[j] > ml[j]) lev[j] = ml[j];
+    __syncwarp();
+  }
   int8_t* mrow = map_ws + (long long)row * a.Nk;
   for (int j = lane; j < a.Nk; j += 32) {
     mrow[j] = lev[j];
@@ -671,7 +682,8 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 32 * rows_per_cta, smem, st>>>(
-        a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (int8_t*)(ws + L.map), user_map,
+        a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (const int8_t*)(ws + L.maxlev),
+        (int8_t*)(ws + L.map), user_map,
         block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
     return cudaGetLastError();
   };

@@ -29,6 +29,7 @@ psa_status_t validate(const psa_params_t* p) {
   if (p->causal != 0 && p->causal != 1) return PSA_ERR_INVALID_ARG;
   if (p->assign != PSA_ASSIGN_THRESHOLD && p->assign != PSA_ASSIGN_QUANTILE) return PSA_ERR_INVALID_ARG;
   if (p->forced_prefix_tokens < 0) return PSA_ERR_INVALID_ARG;
+  if (!(p->sim_threshold <= 1.f)) return PSA_ERR_INVALID_ARG;             // also rejects NaN
   if (p->d != 64 && p->d != 128) return PSA_ERR_UNSUPPORTED;
   if (p->kv_blk != 64) return PSA_ERR_UNSUPPORTED;
   if (p->q_blk != 64 && p->q_blk != 128) return PSA_ERR_UNSUPPORTED;
@@ -63,7 +64,10 @@ psa_status_t check_ptrs(std::initializer_list<const void*> required) {
 
 psa_status_t run_pyramid(const psa_params_t* p, const Layout& L, const void* K, const void* V,
                          void* ws, cudaStream_t st) {
-  return from_cuda(launch_pyramid(*p, L, K, V, (char*)ws, st));
+  psa_status_t r = from_cuda(launch_pyramid(*p, L, K, V, (char*)ws, st));
+  if (r == PSA_OK && p->sim_threshold > -1.f)
+    r = from_cuda(launch_similarity(*p, L, K, (char*)ws, st));
+  return r;
 }
 
 psa_status_t run_mask(const psa_params_t* p, const Layout& L, const void* Q, void* ws,

@@ -29,6 +29,7 @@ struct Layout {
   size_t qmh, qml;            // query-block means [B, Hq, Nq, d]
   size_t zlog;                // block logits fp32 [B, Hq, Nq, Nk]
   size_t map;                 // internal level map int8 [B, Hq, Nq, Nk]
+  size_t maxlev;              // int8 [B, Hkv, Nk]: largest level the cosine constraint allows
   size_t counts;              // int4 per query block: entries at level 0..3
   size_t list;                // int32 [B, Hq, Nq, Nk]: KV block indices, by level then index
   size_t total;
@@ -59,6 +60,7 @@ inline __host__ __device__ Layout make_layout(const psa_params_t& p) {
   L.qml = off; off += align256(rowsq * p.d * 4);
   L.zlog = off; off += align256(rowsq * L.Nk * 4);
   L.map = off; off += align256(rowsq * L.Nk);
+  L.maxlev = off; off += align256((size_t)p.B * p.Hkv * L.Nk);
   L.counts = off; off += align256(rowsq * 16);
   L.list = off; off += align256(rowsq * L.Nk * 4);
   L.total = off;
@@ -70,6 +72,7 @@ struct MaskArgs {
   int B, Hq, Hkv, N, d, q_blk, kv_blk, Nq, Nk;
   int causal, forced_prefix_tokens;
   int assign;                 // psa_assign_t
+  float sim_threshold;        // cosine constraint; <= -1: off
   float scale;
   float tau[kLevels];
 };
@@ -80,6 +83,7 @@ inline MaskArgs make_mask_args(const psa_params_t& p, const Layout& L, float sca
   a.q_blk = p.q_blk; a.kv_blk = p.kv_blk; a.Nq = L.Nq; a.Nk = L.Nk;
   a.causal = p.causal; a.forced_prefix_tokens = p.forced_prefix_tokens;
   a.assign = (int)p.assign;
+  a.sim_threshold = p.sim_threshold;
   a.scale = scale;
   for (int l = 0; l < kLevels; ++l) a.tau[l] = p.tau[l];
   return a;
@@ -113,6 +117,8 @@ __device__ __forceinline__ uint64_t global_ns() {
 namespace psa {
 cudaError_t launch_pyramid(const psa_params_t& p, const Layout& L, const void* K, const void* V,
                            char* ws, cudaStream_t st);
+cudaError_t launch_similarity(const psa_params_t& p, const Layout& L, const void* K, char* ws,
+                              cudaStream_t st);
 cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, char* ws,
                          cudaStream_t st);
 cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, char* ws,

@@ -1,0 +1,113 @@
+// Cosine-similarity constraint on the pyramid levels.
+//
+// The top168.com article on PSA (ablations) names a cosine-similarity
+// constraint on mask generation and its gain, without defining it.  The
+// library's reading: every pooled row of level l >= 1 merges two rows of
+// level l - 1 (token ranges [2g f, (2g+1) f) and [(2g+1) f, (2g+2) f) with
+// f = 2^(l-1), cut at N); the merge is similar when the cosine of the two
+// halves' mean keys is >= theta (an empty or zero half passes).  KV block j
+// may be represented at level l when every merge at levels 1..l inside it is
+// similar; the assignment lowers kept levels above that.
+//
+// One warp per (batch, KV head, KV block); lane = d/32 columns.  Every merge
+// lies inside one 8-token group, so the block is walked group by group: the
+// 7 merges of a group (4 at level 1, 2 at level 2, 1 at level 3) need 21
+// partial sums (a . b, |a|^2, |b|^2), reduced across the warp together.  The
+// cosine is taken of the halves' sums (same direction as their means) in fp32.
+#include "psa_internal.cuh"
+
+namespace psa {
+namespace {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K,
+                                                         int8_t* __restrict__ maxlev, int N,
+                                                         int Nk, long long n_items, float theta) {
+  constexpr int CPL = D / 32;                  // columns per lane
+  const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= n_items) return;                 // whole warp
+  const int j = (int)(item % Nk);
+  const long long bh = item / Nk;
+  const T* base = K + (bh * N) * D + lane * CPL;
+  bool ok1 = true, ok2 = true, ok3 = true;
+  for (int g8 = 0; g8 < 8; ++g8) {
+    const int t0 = j * 64 + g8 * 8;
+    if (t0 >= N) break;
+    const int nv = min(8, N - t0);             // valid tokens of this group
+    float x[8][CPL];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) x[t][c] = t < nv ? to_f32(base[(long long)(t0 + t) * D + c]) : 0.f;
+    // halves of the 7 merges as sums of tokens: level 1 (2p | 2p+1),
+    // level 2 (4q, 4q+1 | 4q+2, 4q+3), level 3 (0..3 | 4..7)
+    float part[21];
+#pragma unroll
+    for (int i = 0; i < 21; ++i) part[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      float s2[4], s4[2];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = x[2 * q][c], b = x[2 * q + 1][c];
+        part[3 * q] = fmaf(a, b, part[3 * q]);
+        part[3 * q + 1] = fmaf(a, a, part[3 * q + 1]);
+        part[3 * q + 2] = fmaf(b, b, part[3 * q + 2]);
+        s2[q] = a + b;
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float a = s2[2 * q], b = s2[2 * q + 1];
+        part[12 + 3 * q] = fmaf(a, b, part[12 + 3 * q]);
+        part[13 + 3 * q] = fmaf(a, a, part[13 + 3 * q]);
+        part[14 + 3 * q] = fmaf(b, b, part[14 + 3 * q]);
+        s4[q] = a + b;
+      }
+      part[18] = fmaf(s4[0], s4[1], part[18]);
+      part[19] = fmaf(s4[0], s4[0], part[19]);
+      part[20] = fmaf(s4[1], s4[1], part[20]);
+    }
+#pragma unroll
+    for (int i = 0; i < 21; ++i)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+    // merge m (level l, second half starting at token `second`) exists when
+    // that token exists; cos >= theta, with a zero half passing
+    auto similar = [&](int m) {
+      const float nn = part[3 * m + 1] * part[3 * m + 2];
+      return nn == 0.f || part[3 * m] >= theta * sqrtf(nn);
+    };
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (2 * q + 1 < nv && !similar(q)) ok1 = false;
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      if (4 * q + 2 < nv && !similar(4 + q)) ok2 = false;
+    if (4 < nv && !similar(6)) ok3 = false;
+  }
+  if (lane == 0) maxlev[item] = (int8_t)(ok1 ? (ok2 ? (ok3 ? 3 : 2) : 1) : 0);
+}
+
+template <typename T, int D>
+cudaError_t similarity_typed(const psa_params_t& p, const Layout& L, const void* K, char* ws,
+                             cudaStream_t st) {
+  const long long n_items = (long long)p.B * p.Hkv * L.Nk;
+  const long long blocks = (n_items + 7) / 8;
+  similarity_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+      (const T*)K, (int8_t*)(ws + L.maxlev), p.N, L.Nk, n_items, p.sim_threshold);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_similarity(const psa_params_t& p, const Layout& L, const void* K, char* ws,
+                              cudaStream_t st) {
+  if (p.dtype == PSA_BF16)
+    return p.d == 128 ? similarity_typed<__nv_bfloat16, 128>(p, L, K, ws, st)
+                      : similarity_typed<__nv_bfloat16, 64>(p, L, K, ws, st);
+  return p.d == 128 ? similarity_typed<float, 128>(p, L, K, ws, st)
+                    : similarity_typed<float, 64>(p, L, K, ws, st);
+}
+
+}  // namespace psa

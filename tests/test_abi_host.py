@@ -94,6 +94,15 @@ def test_selftest_argument_errors_before_any_launch():
     assert P.lib().psa_selftest_wait_timeout(ctypes.byref(bad), B, need, 1000, None) == 1
 
 
+def test_similarity_threshold_validated():
+    """The cosine threshold: NaN or above 1 is rejected; -1 and below turn the
+    constraint off and are valid."""
+    for t in (-5.0, -1.0, 0.0, 0.95, 1.0):
+        assert P.workspace_size(P.make_params(1, 2, 2, 1024, 64, sim_threshold=t)) > 0, t
+    for t in (float("nan"), 1.0001, float("inf")):
+        assert P.workspace_size(P.make_params(1, 2, 2, 1024, 64, sim_threshold=t)) == 0, t
+
+
 def test_assign_rule_validated():
     p = P.make_params(1, 2, 2, 1024, 64, assign=P.ASSIGN_QUANTILE)
     assert P.workspace_size(p) > 0
