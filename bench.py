@@ -66,11 +66,11 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "0b19d19577369894"): 469.531904e6 + 90.338304e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "df1ce9ed2e423f8f"): 471.304704e6 + 91.282176e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
-BWD_TRAFFIC = {("wan2.1_1.3b", 12, "1fe079a7827458c7"): 1888.015104e6 + 1349.937920e6}
+BWD_TRAFFIC = {("wan2.1_1.3b", 12, "c53780ce1a52910b"): 1842.916608e6 + 1340.378624e6}
 
 
 def attn_source_hash(sources=ATTN_SOURCES) -> str:

@@ -9,37 +9,63 @@
 // may be represented at level l when every merge at levels 1..l inside it is
 // similar; the assignment lowers kept levels above that.
 //
-// One warp per (batch, KV head, KV block); lane = d/32 columns.  Every merge
-// lies inside one 8-token group, so the block is walked group by group: the
-// 7 merges of a group (4 at level 1, 2 at level 2, 1 at level 3) need 21
-// partial sums (a . b, |a|^2, |b|^2), reduced across the warp together.  The
-// cosine is taken of the halves' sums (same direction as their means) in fp32.
+// One CTA per (batch, KV head, KV block), one warp per 8-token group (every
+// merge lies inside one group); lane = d/32 columns.  A group's 7 merges (4
+// at level 1, 2 at level 2, 1 at level 3) need 21 partial sums (a . b,
+// |a|^2, |b|^2), reduced across the warp together; the warps' verdicts are
+// combined per level with a block-wide AND.  The cosine is taken of the
+// halves' sums (same direction as their means) in fp32.
 #include "psa_internal.cuh"
 
 namespace psa {
 namespace {
 
+// N consecutive elements (a lane's columns of one token) as fp32, one vector load.
+template <int N> __device__ __forceinline__ void load_cols(const __nv_bfloat16* p, float* x) {
+  if constexpr (N == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    x[0] = a.x; x[1] = a.y;
+  }
+}
+template <int N> __device__ __forceinline__ void load_cols(const float* p, float* x) {
+  if constexpr (N == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K,
                                                          int8_t* __restrict__ maxlev, int N,
-                                                         int Nk, long long n_items, float theta) {
+                                                         int Nk, float theta) {
   constexpr int CPL = D / 32;                  // columns per lane
-  const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (item >= n_items) return;                 // whole warp
+  const long long item = blockIdx.x;           // (b * Hkv + h) * Nk + j
   const int j = (int)(item % Nk);
   const long long bh = item / Nk;
-  const T* base = K + (bh * N) * D + lane * CPL;
+  const int lane = threadIdx.x & 31, g8 = threadIdx.x >> 5;
+  const int t0 = j * 64 + g8 * 8;
+  const int nv = max(0, min(8, N - t0));       // valid tokens of this warp's group
   bool ok1 = true, ok2 = true, ok3 = true;
-  for (int g8 = 0; g8 < 8; ++g8) {
-    const int t0 = j * 64 + g8 * 8;
-    if (t0 >= N) break;
-    const int nv = min(8, N - t0);             // valid tokens of this group
+  if (nv > 1) {                                // whole warp; a single token merges nothing
+    const T* base = K + (bh * N + t0) * D + lane * CPL;
     float x[8][CPL];
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
+    for (int t = 0; t < 8; ++t) {
+      if (t < nv) {
+        load_cols<CPL>(base + (long long)t * D, x[t]);
+      } else {
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) x[t][c] = t < nv ? to_f32(base[(long long)(t0 + t) * D + c]) : 0.f;
+        for (int c = 0; c < CPL; ++c) x[t][c] = 0.f;
+      }
+    }
     // halves of the 7 merges as sums of tokens: level 1 (2p | 2p+1),
     // level 2 (4q, 4q+1 | 4q+2, 4q+3), level 3 (0..3 | 4..7)
     float part[21];
@@ -72,8 +98,8 @@ __global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K
     for (int i = 0; i < 21; ++i)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
-    // merge m (level l, second half starting at token `second`) exists when
-    // that token exists; cos >= theta, with a zero half passing
+    // merge m exists when its second half holds a token; cos >= theta, with
+    // a zero half passing
     auto similar = [&](int m) {
       const float nn = part[3 * m + 1] * part[3 * m + 2];
       return nn == 0.f || part[3 * m] >= theta * sqrtf(nn);
@@ -86,16 +112,18 @@ __global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K
       if (4 * q + 2 < nv && !similar(4 + q)) ok2 = false;
     if (4 < nv && !similar(6)) ok3 = false;
   }
-  if (lane == 0) maxlev[item] = (int8_t)(ok1 ? (ok2 ? (ok3 ? 3 : 2) : 1) : 0);
+  ok1 = __syncthreads_and(ok1);
+  ok2 = __syncthreads_and(ok2);
+  ok3 = __syncthreads_and(ok3);
+  if (threadIdx.x == 0) maxlev[item] = (int8_t)(ok1 ? (ok2 ? (ok3 ? 3 : 2) : 1) : 0);
 }
 
 template <typename T, int D>
 cudaError_t similarity_typed(const psa_params_t& p, const Layout& L, const void* K, char* ws,
                              cudaStream_t st) {
   const long long n_items = (long long)p.B * p.Hkv * L.Nk;
-  const long long blocks = (n_items + 7) / 8;
-  similarity_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
-      (const T*)K, (int8_t*)(ws + L.maxlev), p.N, L.Nk, n_items, p.sim_threshold);
+  similarity_kernel<T, D><<<(unsigned)n_items, 256, 0, st>>>(
+      (const T*)K, (int8_t*)(ws + L.maxlev), p.N, L.Nk, p.sim_threshold);
   return cudaGetLastError();
 }
 
