@@ -12,8 +12,8 @@
 // One CTA per (batch, KV head, KV block), one warp per 8-token group (every
 // merge lies inside one group); lane = d/32 columns.  A group's 7 merges (4
 // at level 1, 2 at level 2, 1 at level 3) need 21 partial sums (a . b,
-// |a|^2, |b|^2), reduced across the warp together; the warps' verdicts are
-// combined per level with a block-wide AND.  The cosine is taken of the
+// |a|^2, |b|^2), reduced across the warp by one reduce-scatter; the warps'
+// verdicts are combined per level with a block-wide AND.  The cosine is taken of the
 // halves' sums (same direction as their means) in fp32.
 #include "psa_internal.cuh"
 
@@ -68,9 +68,9 @@ __global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K
     }
     // halves of the 7 merges as sums of tokens: level 1 (2p | 2p+1),
     // level 2 (4q, 4q+1 | 4q+2, 4q+3), level 3 (0..3 | 4..7)
-    float part[21];
+    float part[32];                            // 21 used, padded for the reduction below
 #pragma unroll
-    for (int i = 0; i < 21; ++i) part[i] = 0.f;
+    for (int i = 0; i < 32; ++i) part[i] = 0.f;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
       float s2[4], s4[2];
@@ -94,16 +94,28 @@ __global__ void __launch_bounds__(256) similarity_kernel(const T* __restrict__ K
       part[19] = fmaf(s4[0], s4[0], part[19]);
       part[20] = fmaf(s4[1], s4[1], part[20]);
     }
+    // reduce-scatter across the warp: at each step a lane keeps the half of
+    // its values that its lane bit selects and adds its partner's copy of
+    // that half; at the end lane i holds the warp's sum of value i (31
+    // shuffles for all 32 values)
 #pragma unroll
-    for (int i = 0; i < 21; ++i)
+    for (int o = 16; o > 0; o >>= 1) {
+      const bool upper = lane & o;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
-    // merge m exists when its second half holds a token; cos >= theta, with
-    // a zero half passing
-    auto similar = [&](int m) {
-      const float nn = part[3 * m + 1] * part[3 * m + 2];
-      return nn == 0.f || part[3 * m] >= theta * sqrtf(nn);
-    };
+      for (int i = 0; i < o; ++i) {
+        const float send = upper ? part[i] : part[i + o];
+        const float keep = upper ? part[i + o] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    // merge m: a . b on lane 3m, |a|^2 and |b|^2 on lanes 3m + 1, 3m + 2;
+    // cos >= theta, with a zero half passing
+    const float na = __shfl_down_sync(0xffffffffu, part[0], 1);
+    const float nb = __shfl_down_sync(0xffffffffu, part[0], 2);
+    const float nn = na * nb;
+    const unsigned sim = __ballot_sync(0xffffffffu, nn == 0.f || part[0] >= theta * sqrtf(nn));
+    auto similar = [&](int m) { return (sim >> (3 * m)) & 1u; };
+    // merge m exists when its second half holds a token
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       if (2 * q + 1 < nv && !similar(q)) ok1 = false;
