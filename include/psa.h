@@ -244,6 +244,9 @@ size_t psa_backward_workspace_size(const psa_params_t* params);
  *    bytes; caller-owned scratch, overwritten.
  *  dQ [B, Hq, N, d], dK, dV [B, Hkv, N, d]: device outputs in the input dtype,
  *    16-byte aligned; every element is written.
+ * dQ is deterministic.  dK and dV are summed in fp32 with atomic adds (a pooled
+ * row collects from every query block that keeps it), whose order varies, so
+ * repeated calls agree to rounding, not bit for bit.
  * Asynchronous on `stream`.  Errors as psa_forward (PSA_ERR_INVALID_ARG for a
  * NULL lse or bwd_workspace). */
 psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void* K, const void* V,

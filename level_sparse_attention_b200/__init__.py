@@ -249,6 +249,48 @@ def psa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_blk: int = 
     return (O, lse, lm) if return_map else (O, lse)
 
 
+class _PSAFunction(torch.autograd.Function):
+    """psa_forward in the forward pass; psa_backward, on the map the forward
+    pass chose (held fixed), in the backward pass."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, q_blk, kv_blk, tau, causal, forced_prefix_tokens, scale, assign,
+                sim_threshold):
+        B, Hq, N, d = q.shape
+        p = make_params(B, Hq, k.shape[1], N, d, q_blk, kv_blk, tau, causal,
+                        forced_prefix_tokens, scale, q.dtype, assign, sim_threshold)
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        ws = new_workspace(p, q.device)
+        O = torch.empty_like(q)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+        lm = torch.empty(map_shape(p), dtype=torch.int8, device=q.device)
+        forward(p, q, k, v, O, ws, lse, lm)
+        ctx.save_for_backward(q, k, v, O, lse, lm)
+        ctx.p = p
+        return O
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, O, lse, lm = ctx.saved_tensors
+        p = ctx.p
+        ws = new_workspace(p, q.device)
+        bws = new_backward_workspace(p, q.device)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        backward(p, q, k, v, O, lse, dO.contiguous(), ws, bws, dq, dk, dv, level_map=lm)
+        return dq, dk, dv, None, None, None, None, None, None, None, None
+
+
+def psa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_blk: int = 128,
+                  kv_blk: int = 64, tau: Sequence[float] = (0.6, 0.8, 0.9, 0.97),
+                  causal: bool = False, forced_prefix_tokens: int = 0, scale: float = 0.0,
+                  assign: int = ASSIGN_THRESHOLD, sim_threshold: float = -1.0) -> torch.Tensor:
+    """PSA attention O [B, Hq, N, d] of CUDA tensors q [B, Hq, N, d], k/v
+    [B, Hkv, N, d] (bf16 or fp32), differentiable: the backward pass runs
+    psa_backward on the level map the forward pass chose."""
+    return _PSAFunction.apply(q, k, v, q_blk, kv_blk, tuple(float(t) for t in tau), causal,
+                              forced_prefix_tokens, scale, assign, sim_threshold)
+
+
 def head_shard(Hq: int, Hkv: int, rank: int, world: int) -> Tuple[int, int, int, int]:
     """The heads rank `rank` of `world` takes of one problem: query heads
     [q0, q1) and the KV heads [kv0, kv1) they read (query head h reads KV

@@ -238,3 +238,29 @@ def test_backward_full_size_sampled(name):
     others = [h for h in range(w.Hkv) if h not in kv_heads]
     if others:
         assert bool((gk[0, others] == 0).all()) and bool((gv[0, others] == 0).all())
+
+
+def test_autograd_entry_point_matches_direct_calls():
+    """psa_attention: O and dQ equal psa_forward's and psa_backward's on the
+    same map, bit for bit.  dK and dV are sums by float atomics, whose order
+    varies between calls, so they agree to rounding: within one bf16 ulp after
+    the final rounding."""
+    w = CASES["bf16_gqa_causal"]
+    inp = W.make_inputs(w)
+    tau = W.thresholds(w)
+    q, k, v = (G.to_device(x, w.dtype) for x in (inp.q, inp.k, inp.v))
+    qg, kg, vg = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = P.psa_attention(qg, kg, vg, w.q_blk, w.kv_blk, tau, w.causal)
+    dO, _ = _grad_out(w, 11)
+    o.backward(dO)
+    out, lse, lm = P.psa_forward(q, k, v, w.q_blk, w.kv_blk, tau, w.causal, return_map=True)
+    assert torch.equal(o.detach(), out)
+    p = G.params_for(w)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    P.backward(p, q, k, v, out, lse, dO, P.new_workspace(p), P.new_backward_workspace(p),
+               dq, dk, dv, level_map=lm)
+    torch.cuda.synchronize()
+    assert torch.equal(qg.grad, dq)
+    for a, b in ((kg.grad, dk), (vg.grad, dv)):
+        a, b = a.float(), b.float()
+        assert bool(((a - b).abs() <= 2.0 ** -7 * b.abs() + 1e-6 * b.abs().max()).all())
