@@ -106,12 +106,14 @@ def _oracle(w, inp, m, dO64):
     return OB.psa_backward(Q, K, V, dO64, m, w.q_blk, w.kv_blk, w.causal)
 
 
-def compare_grad(got, ref, dtype, what):
-    scale = max(float(np.abs(ref).max()), 1e-30)
+def compare_grad(got, ref, dtype, what, floor=1e-30):
+    """Errors relative to the reference's largest and mean magnitudes (each at
+    least ``floor``, for gradients that vanish in exact arithmetic)."""
+    scale = max(float(np.abs(ref).max()), floor)
     err = np.abs(got - ref)
     assert np.all(np.isfinite(got)), what
     max_rel = float(err.max()) / scale
-    mean_rel = float(err.mean() / max(np.abs(ref).mean(), 1e-30))
+    mean_rel = float(err.mean() / max(np.abs(ref).mean(), floor))
     if dtype == "bf16":
         assert max_rel <= 3e-2 and mean_rel <= 1e-2, (what, max_rel, mean_rel)
     else:
