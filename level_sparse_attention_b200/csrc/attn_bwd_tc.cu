@@ -99,6 +99,26 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// packed fp32 pairs (sm_100 f32x2 instructions)
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -353,41 +373,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         const int* mpos = reinterpret_cast<const int*>(mt + 512);
         const int* mdst = reinterpret_cast<const int*>(mt + 1024);
         {
-          // P and dS of keys [64h, 64h + 64) of row r
-          uint32_t sv[64], gv[64];
-          tmem_ldn<64>(T_S + lane_off + 64 * h, sv);
-          tmem_ldn<64>(T_DP + lane_off + 64 * h, gv);
-          tmem_ld_wait();
-          reg_fence<64>(sv);
-          reg_fence<64>(gv);
-          uint32_t pk[32], xk[32];
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const float4 b4 = *reinterpret_cast<const float4*>(mbias + 64 * h + c);
-            const int4 k4 = *reinterpret_cast<const int4*>(mpos + 64 * h + c);
-            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-            const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
-            float pp[4], xx[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float x = fmaf(__uint_as_float(sv[c + i]), sl2, bb[i]) - lse2;
-              const bool keep = live && qpos >= kk[i];
-              pp[i] = keep ? ex2(x) : 0.f;          // -inf bias (no key) gives 0
-              xx[i] = pp[i] * (__uint_as_float(gv[c + i]) - Di);
-            }
-            pk[c / 2] = pack_bf16(pp[0], pp[1]);
-            pk[c / 2 + 1] = pack_bf16(pp[2], pp[3]);
-            xk[c / 2] = pack_bf16(xx[0], xx[1]);
-            xk[c / 2 + 1] = pack_bf16(xx[2], xx[3]);
-          }
-          // row r, keys [64h, 64h + 64): half h of the P / dS tiles, 128-byte
-          // swizzle (16-byte chunk index XOR row mod 8)
+          // P and dS of keys [64h, 64h + 64) of row r, 32 keys at a time:
+          // x = S * scale * log2e + (log2 c - lse * log2e) in pairs, P = exp2(x)
+          // (a -inf bias, no key, gives 0), dS = P (dP - D), written to half h
+          // of the P / dS tiles (128-byte swizzle: 16-byte chunk index XOR row
+          // mod 8).  A row that kept no key (or lies past N) writes zeros.
+          const uint64_t sl2x2 = f2pack(sl2, sl2), nl2 = f2pack(-lse2, -lse2);
+          const uint64_t nd2 = f2pack(-Di, -Di), zero2 = f2pack(0.f, 0.f);
           const uint32_t rowb = (uint32_t)(h * C::HALF + r * 128);
+#pragma unroll 1
+          for (int q = 0; q < 2; ++q) {
+            uint32_t sv[32], gv[32];
+            tmem_ld32(T_S + lane_off + 64 * h + 32 * q, sv);
+            tmem_ld32(T_DP + lane_off + 64 * h + 32 * q, gv);
+            tmem_ld_wait();
+            reg_fence<32>(sv);
+            reg_fence<32>(gv);
+            uint32_t pk[16], xk[16];
+            if (live) {
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const uint32_t o = rowb + (uint32_t)((cc ^ (r & 7)) << 4);
-            st_shared_v4(sbase + C::OFF_P + o, pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-            st_shared_v4(sbase + C::OFF_DS + o, xk[4 * cc], xk[4 * cc + 1], xk[4 * cc + 2], xk[4 * cc + 3]);
+              for (int c = 0; c < 32; c += 4) {
+                const int k = 64 * h + 32 * q + c;
+                const float4 b4 = *reinterpret_cast<const float4*>(mbias + k);
+                float x[4], pp[4], xx[4];
+                f2unpack(ffma2(f2pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2,
+                               fadd2(f2pack(b4.x, b4.y), nl2)), x[0], x[1]);
+                f2unpack(ffma2(f2pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sl2x2,
+                               fadd2(f2pack(b4.z, b4.w), nl2)), x[2], x[3]);
+                if (p.causal) {
+                  const int4 k4 = *reinterpret_cast<const int4*>(mpos + k);
+                  if (qpos < k4.x) x[0] = -INFINITY;
+                  if (qpos < k4.y) x[1] = -INFINITY;
+                  if (qpos < k4.z) x[2] = -INFINITY;
+                  if (qpos < k4.w) x[3] = -INFINITY;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pp[i] = ex2(x[i]);
+#pragma unroll
+                for (int i = 0; i < 4; i += 2) {
+                  const uint64_t gd = fadd2(f2pack(__uint_as_float(gv[c + i]), __uint_as_float(gv[c + i + 1])), nd2);
+                  f2unpack(ffma2(f2pack(pp[i], pp[i + 1]), gd, zero2), xx[i], xx[i + 1]);
+                }
+                pk[c / 2] = pack_bf16(pp[0], pp[1]);
+                pk[c / 2 + 1] = pack_bf16(pp[2], pp[3]);
+                xk[c / 2] = pack_bf16(xx[0], xx[1]);
+                xk[c / 2 + 1] = pack_bf16(xx[2], xx[3]);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = xk[i] = 0u;
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint32_t o = rowb + (uint32_t)(((4 * q + cc) ^ (r & 7)) << 4);
+              st_shared_v4(sbase + C::OFF_P + o, pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+              st_shared_v4(sbase + C::OFF_DS + o, xk[4 * cc], xk[4 * cc + 1], xk[4 * cc + 2], xk[4 * cc + 3]);
+            }
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
