@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.n_rows;
+  const Schedule sched = make_schedule(n_items, p.Nq, p.causal != 0);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -197,7 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     int gk = 0, iq = 0;
     bool ok = true;
     int* lcache = reinterpret_cast<int*>(smem + C::OFF_LIST + (kprod ? 0 : kListCache * 4));
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    for (int jb = 0; ok && jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
       const RowWork w = row_work(p.counts[item]);
       const int T = w.tiles;
       if (T == 0) continue;
@@ -294,7 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
       constexpr uint32_t kRow16 = (16 * 128) >> 4;   // 16 rows along K of an MN-major view
       bool ok = true;
       int u = 0, iq = 0;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+      for (int jb = 0; ok && jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
         if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
@@ -352,7 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     const float sl2 = p.scale_log2;
     int u = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    for (int jb = 0; jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int bhk = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / (p.Hq / p.Hkv);

@@ -150,9 +150,9 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 // polynomial above, the rest the transcendental unit (MUFU).
 constexpr int kPolyPairs = 0;
 
-// Items (query blocks) of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
-// Consecutive CTAs take consecutive query blocks of the same head, so the
-// head's K/V and pyramid stay in L2 while its query blocks are processed.
+// Items (query blocks) of this CTA: the bands of tile::Schedule (round robin
+// over consecutive query blocks of a head, for L2 reuse of its K/V; causally,
+// longest rows first, dealt in a snake so that the CTAs' loads even out).
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.n_rows;
+  const Schedule sched = make_schedule(n_items, p.Nq, p.causal != 0);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -221,7 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ---------------------------------------------------- K / Q producer
     int gk = 0, iq = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    for (int jb = 0; ok && jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
       const RowWork w = row_work(p.counts[item]);
       const int T = w.tiles;
       if (T == 0) continue;
@@ -319,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ V producer
     int gv = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    for (int jb = 0; ok && jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
       const RowWork w = row_work(p.counts[item]);
       const int T = w.tiles;
       if (T == 0) continue;
@@ -396,7 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       };
       // Per query block: QK(0), QK(1); then for each tile t: PV(t), QK(t + 2).
       int g = 0, iq = 0;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+      for (int jb = 0; ok && jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
         if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
@@ -445,7 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint64_t sc2 = f2pack(sc, sc);
     int g = 0, ns = 0, nb = 0;               // tiles before this block, stream tiles, blocks with work
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    for (int jb = 0; jb < sched.bands(); ++jb) {
+      const int item = sched.item(jb);
+      if (item < 0) continue;
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int qpos = qa * kBM + r;

@@ -69,5 +69,42 @@ __device__ __forceinline__ TileEntry tile_entry(const RowWork& w, const int* lro
   return te;
 }
 
+// The query blocks (items, (b * Hq + h) * Nq + a) a persistent CTA c of G
+// processes, band by band: band j holds positions [j G, j G + G).  Without
+// causality every row costs about the same, and CTA c takes position j G + c
+// = the item itself, so that consecutive CTAs work on consecutive query
+// blocks of a head while its K/V stay in L2.  Causally, row a keeps about
+// a + 1 blocks' worth of keys: positions are dealt in a snake (band j goes
+// c or G - 1 - c alternately) and position p is query block Nq - 1 - p / BH
+// of head p % BH, so every band holds rows of about the same length and the
+// bands go from the longest rows to the shortest.  Every role of a CTA walks
+// the same sequence.
+struct Schedule {
+  int G, c, n, Nq, BH;
+  bool causal;
+  __device__ __forceinline__ int bands() const { return (n + G - 1) / G; }
+  // the item of band j, or -1 where the band has none for this CTA
+  __device__ __forceinline__ int item(int j) const {
+    if (!causal) {
+      const int k = j * G + c;
+      return k < n ? k : -1;
+    }
+    const int pos = j * G + ((j & 1) ? G - 1 - c : c);
+    if (pos >= n) return -1;
+    return (pos % BH) * Nq + (Nq - 1 - pos / BH);
+  }
+};
+
+__device__ __forceinline__ Schedule make_schedule(int n_items, int Nq, bool causal) {
+  Schedule s;
+  s.G = gridDim.x;
+  s.c = blockIdx.x;
+  s.n = n_items;
+  s.Nq = Nq;
+  s.BH = n_items / Nq;
+  s.causal = causal;
+  return s;
+}
+
 }  // namespace tile
 }  // namespace psa
