@@ -66,11 +66,11 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "df1ce9ed2e423f8f"): 471.304704e6 + 91.282176e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "3fcecd4c344d457b"): 470.370304e6 + 90.855424e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
-BWD_TRAFFIC = {("wan2.1_1.3b", 12, "c53780ce1a52910b"): 1842.916608e6 + 1340.378624e6}
+BWD_TRAFFIC = {("wan2.1_1.3b", 12, "95d97592c8425313"): 1894.116096e6 + 1364.966144e6}
 
 
 def attn_source_hash(sources=ATTN_SOURCES) -> str:

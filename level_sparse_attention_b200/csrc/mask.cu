@@ -28,10 +28,11 @@ namespace {
 
 // -------------------------------------------------------------- q means
 
-// One CTA of 256 threads per query block.  Thread t takes the 8-column chunk
-// t % (d/8) of rows t / (d/8) + k * 256/(d/8) (at most 8 rows: q_blk <= 128,
-// d >= 64) and issues all its loads before adding.  Lanes holding the same
-// chunk are summed with shuffles, the 8 warps' partial sums in shared memory.
+// One CTA of q_blk * d / 64 threads per query block (256 for 128 x 128, 128
+// for 128 x 64 or 64 x 128): thread t takes the 8-column chunk t % (d/8) of
+// rows t / (d/8) + k * parts (parts = threads / (d/8), k < 8), so that every
+// thread issues 8 loads, all before adding.  Lanes holding the same chunk are
+// summed with shuffles, the warps' partial sums in shared memory.
 template <typename T> struct QVec;
 template <> struct QVec<__nv_bfloat16> {
   uint4 raw;
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
   const int lo = qa * a.q_blk;
   const int n = min(a.q_blk, a.N - lo);
   const int chunks = a.d / 8;               // 16 or 8
-  const int parts = 256 / chunks;           // rows read side by side: 16 or 32
+  const int parts = blockDim.x / chunks;    // rows read side by side
   const int c = threadIdx.x % chunks;
   const int part = threadIdx.x / chunks;
   const T* base = Q + (bh * a.N + lo) * a.d + c * 8;
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
     for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
   __shared__ float red[8][16][8];           // [warp][chunk][column]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
   if (lane < chunks)
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[warp][lane][e] = acc[e];
@@ -98,8 +100,7 @@ __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restr
     float sum[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) sum[e] = red[0][c][e];
-#pragma unroll
-    for (int w = 1; w < 8; ++w)
+    for (int w = 1; w < nwarps; ++w)
 #pragma unroll
       for (int e = 0; e < 8; ++e) sum[e] += red[w][c][e];
     // the mean in fp32, stored as tf32 head + exact tail
@@ -657,12 +658,13 @@ cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, 
                          cudaStream_t st) {
   const MaskArgs a = make_mask_args(p, L, 0.f);
   const int grid = p.B * p.Hq * L.Nq;
+  const int threads = p.q_blk * p.d / 64;  // 8 rows per thread: 64 to 256 threads
   float* qh = (float*)(ws + L.qmh);
   float* ql = (float*)(ws + L.qml);
   if (p.dtype == PSA_BF16)
-    qmean_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, (const __nv_bfloat16*)Q, qh, ql);
+    qmean_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(a, (const __nv_bfloat16*)Q, qh, ql);
   else
-    qmean_kernel<float><<<grid, 256, 0, st>>>(a, (const float*)Q, qh, ql);
+    qmean_kernel<float><<<grid, threads, 0, st>>>(a, (const float*)Q, qh, ql);
   return cudaGetLastError();
 }
 
