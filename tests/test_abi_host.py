@@ -79,6 +79,26 @@ def test_argument_errors_before_any_launch():
     assert P.lib().psa_forward(ctypes.byref(p), A, A, A, A, mis4, None, B, need, None) == 3
 
 
+def test_backward_argument_errors_before_any_launch():
+    """psa_backward validates everything on the host before any launch: a
+    NULL lse or scratch, a misaligned lse, scratch or tensor, scratch that is
+    too small, and the forward workspace's own checks."""
+    p = P.make_params(1, 4, 2, 1024, 64)
+    need, bneed = P.workspace_size(p), P.backward_workspace_size(p)
+    assert bneed > 0 and P.backward_workspace_size(P.make_params(1, 4, 2, 1024, 96)) == 0
+    A, W, BW = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    f = lambda lse=A, bws=BW, bbytes=bneed, ws=W, wbytes=need, dq=A: P.lib().psa_backward(
+        ctypes.byref(p), A, A, A, A, lse, A, None, ws, wbytes, bws, bbytes, dq, A, A, None)
+    assert f(lse=None) == 1                                   # lse is required
+    assert f(bws=None) == 1                                   # so is the scratch
+    assert f(lse=ctypes.c_void_p(0x10002)) == 3               # lse: 4-byte alignment
+    assert f(bws=ctypes.c_void_p(0x30010)) == 3               # scratch: 256-byte alignment
+    assert f(bbytes=bneed - 1) == 4                           # scratch too small
+    assert f(wbytes=need - 1) == 4                            # forward workspace too small
+    assert f(dq=ctypes.c_void_p(0x10008)) == 3                # dQ: 16-byte alignment
+    assert f(dq=None) == 1
+
+
 def test_selftest_argument_errors_before_any_launch():
     p = P.make_params(1, 2, 2, 1024, 64)
     need = P.workspace_size(p)
