@@ -30,7 +30,9 @@
 //          of the key's level and pooled row (vector atomics; a pooled row
 //          is shared by every query block that keeps it)
 // At the end of the query block dQ * s is read from TMEM and stored.
-// TMEM columns: S / dK_t [0, 128), dP / dV_t [128, 256), dQ [256, 256 + d).
+// TMEM columns: S / dK_t [0, 128), dP [128, 256), dQ [256, 256 + d),
+// dV_t [384, 384 + d).  dP of the next tile of a block is issued as soon as
+// the softmax has read this tile's, so it overlaps this tile's epilogue.
 // Every mbarrier wait is bounded: on expiry the kernel records a timeout in
 // the workspace error word and winds down without trapping.
 #include "bwd_internal.cuh"
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t T_S = tmem, T_DP = tmem + 128, T_DQ = tmem + 256;
+  const uint32_t T_S = tmem, T_DP = tmem + 128, T_DQ = tmem + 256, T_DV = tmem + 384;
 
   if (warp == 0 || warp == kVWarp) {
     // ----------------------------------------- producers: Q, dO, K (warp 0); V (warp 2)
@@ -303,11 +305,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         const int T = row_work(p.counts[item]).tiles;
         if (T == 0) continue;
         if (!wait_bar(bar(B_QFULL), iq & 1, abort_flag, p.err)) { ok = false; break; }
+        // dP of a tile is issued as soon as its region is free: after the
+        // softmax of the previous tile of the block has read dP (dV_t has
+        // its own columns), so it runs while that tile's epilogue reads
+        // dK_t / dV_t; S waits for the epilogue, since dK_t shares its columns
+        bool dp_issued = false;
+        auto issue_dp = [&](int uu) -> bool {
+          const int sv = uu % KS;
+          if (!wait_bar(bar(B_VFULL + sv), (uu / KS) & 1, abort_flag, p.err)) return false;
+          tc_fence_after();
+          const uint64_t stv = (uint64_t)((sv * C::T_BYTES) >> 4);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t off = (uint64_t)((k >> 2) * kHalfStep + (k & 3) * 2);
+            mma_ss(T_DP, do_k + off, v_k + stv + off, ID_S, k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(B_VEMPTY + sv));
+          return true;
+        };
         for (int t = 0; ok && t < T; ++t, ++u) {
           const int s = u % KS;
           const uint64_t stage = (uint64_t)((s * C::T_BYTES) >> 4);
+          if (!dp_issued && !issue_dp(u)) { ok = false; break; }
           ok = wait_bar(bar(B_KFULL + s), (u / KS) & 1, abort_flag, p.err) &&
-               wait_bar(bar(B_VFULL + s), (u / KS) & 1, abort_flag, p.err) &&
                (u == 0 || wait_bar(bar(B_TFREE), (u - 1) & 1, abort_flag, p.err));
           if (!ok) break;
           tc_fence_after();
@@ -315,10 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           for (int k = 0; k < D / 16; ++k) {
             const uint64_t off = (uint64_t)((k >> 2) * kHalfStep + (k & 3) * 2);
             mma_ss(T_S, q_k + off, k_k + stage + off, ID_S, k > 0 ? 1u : 0u);
-            mma_ss(T_DP, do_k + off, v_k + stage + off, ID_S, k > 0 ? 1u : 0u);
           }
-          mma_commit(bar(B_SFULL));
-          mma_commit(bar(B_VEMPTY + s));
+          mma_commit(bar(B_SFULL));                    // S and dP of tile u
           ok = wait_bar(bar(B_PFULL), u & 1, abort_flag, p.err) &&
                (t > 0 || iq == 0 || wait_bar(bar(B_DQFREE), (iq - 1) & 1, abort_flag, p.err));
           if (!ok) break;
@@ -332,12 +350,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
 #pragma unroll
           for (int k = 0; k < kBM / 16; ++k) {
             const uint64_t roff = (uint64_t)(k * kRow16);
-            mma_ss(T_DP, p_mn + roff, do_mn + roff, ID_KV, k > 0 ? 1u : 0u);
+            mma_ss(T_DV, p_mn + roff, do_mn + roff, ID_KV, k > 0 ? 1u : 0u);
             mma_ss(T_S, ds_mn + roff, q_mn + roff, ID_KV, k > 0 ? 1u : 0u);
           }
           mma_commit(bar(B_GFULL));
           mma_commit(bar(B_KEMPTY + s));
           if (t == T - 1) mma_commit(bar(B_QEMPTY));
+          // the next tile's dP (the softmax of this tile has read dP: PFULL)
+          dp_issued = t + 1 < T;
+          if (dp_issued && !issue_dp(u + 1)) { ok = false; break; }
         }
         ++iq;
       }
@@ -448,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           // epilogue: key r of the tile, columns [h DH, h DH + DH)
           uint32_t kv[DH], vv[DH];
           tmem_ldn<DH>(T_S + lane_off + h * DH, kv);
-          tmem_ldn<DH>(T_DP + lane_off + h * DH, vv);
+          tmem_ldn<DH>(T_DV + lane_off + h * DH, vv);
           tmem_ld_wait();
           reg_fence<DH>(kv);
           reg_fence<DH>(vv);
