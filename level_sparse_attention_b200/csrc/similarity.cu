@@ -13,7 +13,7 @@
 // merge lies inside one group); lane = d/32 columns.  A group's 7 merges (4
 // at level 1, 2 at level 2, 1 at level 3) need 21 partial sums (a . b,
 // |a|^2, |b|^2), reduced across the warp by one reduce-scatter; the warps'
-// verdicts are combined per level with a block-wide AND.  The cosine is taken of the
+// results are combined per level with a block-wide AND.  The cosine is taken of the
 // halves' sums (same direction as their means) in fp32.
 #include "psa_internal.cuh"
 
