@@ -70,7 +70,7 @@ ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "3fcecd4c344d457b"): 470.370304e6 + 90.85542
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
-BWD_TRAFFIC = {("wan2.1_1.3b", 12, "182c3066542407e7"): 1873.167616e6 + 1333.184256e6}
+BWD_TRAFFIC = {("wan2.1_1.3b", 12, "bc04b1e4ab04e483"): 1873.167616e6 + 1333.184256e6}
 
 
 def attn_source_hash(sources=ATTN_SOURCES) -> str:

@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           reg_fence<DH>(kv);
           reg_fence<DH>(vv);
           tc_fence_before();
-          mbar_arrive(bar(B_TFREE));               // S / dP columns free for the next tile
+          mbar_arrive(bar(B_TFREE));               // dK_t, dV_t read: S and dV_t may be overwritten
           const int dst = mdst[r];
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
