@@ -7,5 +7,5 @@ from .psa_oracle import *  # noqa: F401,F403
 from .psa_oracle import (PRUNED, POOL, Pyramid, MaskResult, HeadResult, ForwardResult,
                          cdiv, pool_tokens, build_pyramid, block_rows, query_block_means,
                          block_logits, visible, straddles, rank_blocks, level_of,
-                         apply_overrides, assign_levels, block_max_levels, pyramid_attention, psa_head,
+                         apply_overrides, assign_levels, block_max_levels, correct_map, pyramid_attention, psa_head,
                          psa_forward, executed_flops)

@@ -38,7 +38,7 @@ from typing import Dict, Optional, Sequence
 
 import numpy as np
 
-from .psa_oracle import POOL, block_rows, build_pyramid
+from .psa_oracle import POOL, block_rows, build_pyramid, correct_map
 
 
 def unpool(g: np.ndarray, counts: np.ndarray, f: int, N: int) -> np.ndarray:
@@ -72,9 +72,11 @@ def pyramid_attention_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray,
     the same kept keys as the forward pass (each kept block j's rows of level
     map[a, j], a token mask on causal diagonal blocks), recomputes P, and
     spreads the gradients back to the level rows they came from.  Rows that
-    keep no key have O = 0 and pass no gradient."""
+    keep no key have O = 0 and pass no gradient.  The map is corrected as
+    the forward pass corrects it (``psa_oracle.correct_map``)."""
     N, d = Q.shape
     s = 1.0 / math.sqrt(d) if scale is None else scale
+    level_map, _ = correct_map(level_map, N, bq, bk, causal)
     pyr = build_pyramid(K, V, pool)
     Nq, Nk = level_map.shape
     dQ = np.zeros((N, d), dtype=np.float64)

@@ -18,7 +18,9 @@ Sources (the web pages describing PSA, arXiv:2512.04025):
          adaptive pyramid attention that keeps the probability distribution
          consistent); threshold-based assignment beats quantile-based.
   [skill] "Psa Pyramid Sparse Attention" (skillmd.com), "Core Technique": levels
-         0/1/2/3 are the KV pooled 1x/2x/4x/8x.
+         0/1/2/3 are the KV pooled 1x/2x/4x/8x; "Implementation": sketches of the
+         pooled cache, block scoring, a quantile-style level assignment (top
+         keep-ratio blocks at level 0, the rest in thirds) and the attention.
 
 Where the pages leave a step open, the reading used is stated at the function.
 Every function below works on one (batch, head) slice; ``psa_forward`` loops.
@@ -184,13 +186,34 @@ def quotas(n_visible: int, tau: Sequence[float]) -> np.ndarray:
     """Quantile rule: K_l = ceil(tau_l * n_visible), the number of top-ranked
     blocks at level <= l.  tau is taken at the single precision the C
     interface carries it in, and the product is exact in float64 (a 24-bit
-    significand times an integer below 2^14)."""
+    significand times an integer below 2^14).
+
+    Source: [skill] Implementation, the level-assignment sketch: the top
+    int(n * keep_ratio) blocks by score get level 0 and the rest are cut into
+    thirds for levels 1..3, nothing pruned.  Readings that depart from it:
+      * quotas per level (tau_0..tau_3) instead of one keep ratio and fixed
+        thirds; the sketch is the case tau = (K_0, K_0 + r//3, K_0 + 2r//3, n)/n
+        with K_0 = int(n * keep_ratio), r = n - K_0;
+      * rounded up, not down: a positive tau_0 keeps the top block at level 0,
+        as the threshold rule's exclusive mass does (the sketch's int() gives 0
+        blocks when n * keep_ratio < 1, and its slice of the last 0 sorted
+        indices then selects every block);
+      * blocks ranked at or past K_3 are pruned, so that the rule can be
+        compared with the threshold rule at equal compute (the ablation of
+        [news]); tau_3 = 1 prunes nothing, as the sketch."""
     t = np.asarray(tau, dtype=np.float32).astype(np.float64)
     return np.ceil(t * float(n_visible)).astype(np.int64)
 
 
 def level_of_rank(rank: np.ndarray, K: np.ndarray) -> np.ndarray:
-    """Quantile rule: level = the smallest l with rank < K_l, else pruned (-1)."""
+    """Quantile rule: level = the smallest l with rank < K_l, else pruned (-1).
+    The rank is the block's place in the ranking by P (descending, ties to the
+    lower index), so the blocks past level 0 are cut in order of importance.
+    [skill]'s sketch cuts them in block-index order, which would give level 1
+    to the lowest indices whatever their score, against its own Core
+    Technique (level 1 = medium importance, level 3 = minimal) and [abs]
+    (higher levels for less important blocks); the index order is read as a
+    slip of the sketch."""
     out = np.full(rank.shape, PRUNED, dtype=np.int8)
     for l in reversed(range(len(K))):
         out[rank < K[l]] = l
@@ -296,6 +319,32 @@ def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
 
 # ----------------------------------------------------------------- attention
 
+def correct_map(level_map: np.ndarray, N: int, bq: int, bk: int,
+                causal: bool) -> Tuple[np.ndarray, int]:
+    """A level map as the attention uses it, and how many entries were changed.
+
+    A map handed in by a caller may break the method's contract; the attention
+    never reads future tokens and never reads an undefined level:
+      * a value outside -1..3 is treated as pruned;
+      * causal: a block after the query block's last row is pruned, and a kept
+        block that straddles its diagonal is attended at level 0 with the
+        token mask (a pooled key there would average future tokens; reading:
+        [news] causal and bidirectional paragraph says PSA serves causal
+        generation, and the assignment's own causal overrides do the same).
+    Maps made by ``assign_levels`` already satisfy this and pass unchanged."""
+    lm = np.array(level_map, dtype=np.int64)
+    out = np.where((lm >= -1) & (lm <= 3), lm, PRUNED)
+    if causal:
+        Nq, Nk = out.shape
+        for a in range(Nq):
+            for j in range(Nk):
+                if not visible(a, j, N, bq, bk, True):
+                    out[a, j] = PRUNED
+                elif out[a, j] > 0 and straddles(a, j, N, bq, bk):
+                    out[a, j] = 0
+    return out.astype(np.int8), int((out != lm).sum())
+
+
 def pyramid_attention(Q: np.ndarray, pyr: Pyramid, level_map: np.ndarray, bq: int, bk: int,
                       scale: float, causal: bool = False,
                       pool: Sequence[int] = POOL) -> Tuple[np.ndarray, np.ndarray]:
@@ -308,8 +357,11 @@ def pyramid_attention(Q: np.ndarray, pyr: Pyramid, level_map: np.ndarray, bq: in
     carry the softmax mass of the c_g tokens it averages: it equals attending to
     the pooled key repeated c_g times.  Causal blocks straddling the diagonal
     (always level 0) also mask keys after row i.  A row that keeps no key gets
-    O = 0 and LSE = -inf.  Returns (O [N, d], LSE [N], natural log)."""
+    O = 0 and LSE = -inf.  The map is first put through ``correct_map`` (values
+    outside -1..3 pruned; causally, no future block and no pooled diagonal
+    block).  Returns (O [N, d], LSE [N], natural log)."""
     N, d = Q.shape
+    level_map, _ = correct_map(level_map, N, bq, bk, causal)
     Nq, Nk = level_map.shape
     O = np.zeros((N, d), dtype=np.float64)
     lse = np.full(N, -np.inf, dtype=np.float64)

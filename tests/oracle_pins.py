@@ -236,6 +236,32 @@ def pin_assign_quantile_permutation_and_causal(O):
         assert row[j] == want, (j, rnk, row[j], want)
 
 
+def pin_assign_quantile_listing(O):
+    """The level-assignment sketch of "Psa Pyramid Sparse Attention"
+    (skillmd.com, Implementation), worked by hand in
+    tests/golden/assign_levels_quantile_listing.json: with the stated tau the
+    quantile rule gives the sketch's counts (int(n * keep_ratio) blocks at
+    level 0, the rest in thirds, nothing pruned) with the remainder cut in rank
+    order, not in the sketch's index order; decimal tau whose float32 values
+    lie above K_l / n take one block more; and a quota below one block still
+    keeps the top block at level 0."""
+    with open(os.path.join(GOLDEN, "assign_levels_quantile_listing.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        P = np.array(c["P"], dtype=np.float64)
+        z = np.log(P)[None, :]
+        r = O.assign_levels(z, c["tau"], N=64 * len(P), bq=64, bk=64, rule="quantile")
+        got = r.level_map[0].tolist()
+        assert got == c["levels"], (c["name"], got)
+        if "index_order_levels" in c:
+            n, k0 = c["n"], int(c["n"] * c["keep_ratio"])
+            rest = n - k0
+            want = [k0, rest // 3, 2 * rest // 3 - rest // 3, rest - 2 * rest // 3, 0]
+            have = [got.count(l) for l in (0, 1, 2, 3, -1)]
+            assert have == want, (c["name"], have, want)
+            assert got != c["index_order_levels"]
+
+
 # --------------------------------------------------------------- attention
 
 def _rand_head(seed, N, d):
@@ -354,6 +380,40 @@ def pin_attention_scale_shift(O):
     Q2[:, -1] += 3.0
     out2, _ = O.pyramid_attention(Q2, pyr, lm, bq, bk, 0.4)
     assert np.allclose(out, out2, atol=1e-13)
+
+
+def pin_attention_causal_never_reads_the_future(O):
+    """Causal attention on a caller's map that breaks the contract (future
+    blocks and diagonal blocks at pooled levels, values outside -1..3): row i
+    must not depend on any token after i.  Changing K and V after token t0
+    (inside a diagonal block) leaves rows <= t0 exactly as they were, for
+    every t0 tried; and a value outside -1..3 acts as a pruned block (SDPA
+    with that block masked, the other blocks at level 0)."""
+    N, d, bq, bk = 64 * 6 + 24, 8, 128, 64
+    Q, K, V = _rand_head(31, N, d)
+    rng = np.random.default_rng(32)
+    Nq, Nk = -(-N // bq), -(-N // bk)
+    lm = rng.integers(-1, 4, size=(Nq, Nk)).astype(np.int8)
+    lm[:, -1] = 2                                    # the future of every row but the last
+    lm[1, 2:4] = 3                                   # diagonal blocks of query block 1 pooled
+    lm[2, 4] = 7                                     # out of range
+    pyr = O.build_pyramid(K, V)
+    s = 1 / math.sqrt(d)
+    out, _ = O.pyramid_attention(Q, pyr, lm, bq, bk, s, causal=True)
+    for t0 in (140, 200, 255, 300, 333):
+        K2, V2 = K.copy(), V.copy()
+        K2[t0 + 1:] = rng.standard_normal((N - t0 - 1, d)) * 5.0
+        V2[t0 + 1:] = rng.standard_normal((N - t0 - 1, d)) * 5.0
+        out2, _ = O.pyramid_attention(Q, O.build_pyramid(K2, V2), lm, bq, bk, s, causal=True)
+        assert np.allclose(out2[:t0 + 1], out[:t0 + 1], atol=1e-12, rtol=0), t0
+    # out-of-range values are pruned blocks
+    lmb = np.zeros((Nq, Nk), dtype=np.int8)
+    lmb[0, 1], lmb[2, 3], lmb[3, 0] = 7, -5, 100
+    outb, _ = O.pyramid_attention(Q, pyr, lmb, bq, bk, s)
+    mask = np.zeros((N, N))
+    for a, j in ((0, 1), (2, 3), (3, 0)):
+        mask[a * bq:(a + 1) * bq, j * bk:(j + 1) * bk] = -np.inf
+    assert np.allclose(outb, _sdpa(Q, K, V, mask=mask), atol=1e-12)
 
 
 # --------------------------------------------- cosine-similarity constraint
