@@ -46,7 +46,8 @@ typedef enum {
   PSA_ERR_MISALIGNED = 3,           /* a device pointer breaks its alignment rule       */
   PSA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < psa_workspace_size(params)    */
   PSA_ERR_CUDA = 5,                 /* a CUDA call or launch failed                    */
-  PSA_ERR_DEVICE_TIMEOUT = 6        /* a kernel gave up waiting (see psa_check_device) */
+  PSA_ERR_DEVICE_TIMEOUT = 6,       /* a kernel gave up waiting (see psa_check_device) */
+  PSA_ERR_LEVEL_MAP = 7             /* a caller's level map was corrected (see psa_attention_fwd) */
 } psa_status_t;
 
 typedef enum { PSA_F32 = 0, PSA_BF16 = 1 } psa_dtype_t;
@@ -68,7 +69,12 @@ typedef enum { PSA_ASSIGN_THRESHOLD = 0, PSA_ASSIGN_QUANTILE = 1 } psa_assign_t;
  *                    of the query block's visible KV blocks: the block ranked r
  *                    (0-based) gets the smallest l with r < K_l, K_l =
  *                    ceil(tau[l] * n_visible) computed exactly from the float
- *                    value, else it is pruned.
+ *                    value, else it is pruned.  The level-assignment sketch of
+ *                    "Psa Pyramid Sparse Attention" (Implementation: the top
+ *                    int(n * keep_ratio) blocks at level 0, the rest in thirds,
+ *                    nothing pruned) is the case K = (K_0, K_0 + r/3,
+ *                    K_0 + 2r/3, n), r = n - K_0, with the thirds taken in rank
+ *                    order (the sketch takes them in index order).
  *  causal            1: key position <= query position (blocks after the query
  *                    block are pruned, blocks straddling its diagonal get level
  *                    0 and a token mask).
@@ -147,7 +153,15 @@ psa_status_t psa_score_and_mask(const psa_params_t* params, const void* Q, void*
  * level 0 (the pyramid's other levels come from `workspace`).  level_map:
  * device int8 map to use instead of the one psa_score_and_mask built (NULL =
  * use the workspace's work list); a non-NULL map is turned into a work list
- * in `workspace` first.  O: device [B, Hq, N, d] in dtype.  lse: device fp32
+ * in `workspace` first, held to the contract the mask generator keeps: a
+ * value outside -1..3 counts as pruned, and with causal = 1 a block after the
+ * query block's last row is pruned and a kept block straddling its diagonal
+ * is attended at level 0 with the token mask (a pooled key there would
+ * average future tokens; the top168.com article's causal and bidirectional
+ * paragraph has PSA serve causal generation).  The outputs are those of the
+ * corrected map; if any entry had to be changed, the workspace error word
+ * records it and the next psa_check_device returns PSA_ERR_LEVEL_MAP.
+ * Nothing traps.  O: device [B, Hq, N, d] in dtype.  lse: device fp32
  * [B, Hq, N] natural-log sum of exp of the logits, or NULL.  A row that keeps
  * no key gets O = 0 and lse = -inf. */
 psa_status_t psa_attention_fwd(const psa_params_t* params, const void* Q, const void* K,
@@ -237,7 +251,8 @@ size_t psa_backward_workspace_size(const psa_params_t* params);
  *  level_map: device int8 [B, Hq, Nq, Nk] or NULL.  NULL: the work list the
  *    last forward call left in `workspace` is used (so call this after
  *    psa_forward / psa_attention_fwd with the same workspace); else the list
- *    is rebuilt from the map, as psa_attention_fwd does.
+ *    is rebuilt from the map, as psa_attention_fwd does (with the same
+ *    corrections and PSA_ERR_LEVEL_MAP report).
  *  workspace: the forward workspace, psa_workspace_size(params) bytes; the
  *    pyramid levels in it are rebuilt from K and V.
  *  bwd_workspace: device, 256-byte aligned, psa_backward_workspace_size(params)
@@ -257,7 +272,9 @@ psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void*
 
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
- * check, PSA_ERR_CUDA if the stream reported an error, else PSA_OK. */
+ * check, else PSA_ERR_LEVEL_MAP if a caller's level map was corrected
+ * (psa_attention_fwd, psa_backward), PSA_ERR_CUDA if the stream reported an
+ * error, else PSA_OK. */
 psa_status_t psa_check_device(const psa_params_t* params, void* workspace,
                               size_t workspace_bytes, void* stream);
 

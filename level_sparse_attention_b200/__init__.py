@@ -20,7 +20,8 @@ LIB_PATH = os.path.join(_HERE, "libpsa.so")
 
 F32, BF16 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "misaligned",
-           4: "workspace too small", 5: "CUDA error", 6: "device timeout"}
+           4: "workspace too small", 5: "CUDA error", 6: "device timeout",
+           7: "level map corrected"}
 
 
 class PSAError(RuntimeError):

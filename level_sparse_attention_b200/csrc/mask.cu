@@ -629,19 +629,35 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   emit_list_warp(lev, a.Nk, list + (long long)row * a.Nk, counts + row);
 }
 
+// A caller's level map -> the work list.  The map is held to the method's
+// contract first: a value outside -1..3 counts as pruned; causally, a block
+// after the query block's last row is pruned and a kept block straddling its
+// diagonal is attended at level 0 (with the token mask), since a pooled key
+// there would average future tokens.  Every changed entry sets kErrLevelMap in
+// the workspace error word (psa_check_device reports it).
 __global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
                                    const int8_t* __restrict__ map, int* __restrict__ list,
-                                   int4* __restrict__ counts) {
+                                   int4* __restrict__ counts, int* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * rows_per_cta + warp;
   if (row >= nrows) return;
   const int lev_stride = (a.Nk + 15) & ~15;
   int8_t* lev = reinterpret_cast<int8_t*>(smem) + (size_t)warp * lev_stride;
+  const int q_lo = (row % a.Nq) * a.q_blk;
+  const int q_hi = min(a.N, q_lo + a.q_blk) - 1;
+  bool changed = false;
   for (int j = lane; j < lev_stride; j += 32) {
     const int8_t v = j < a.Nk ? map[(long long)row * a.Nk + j] : (int8_t)-1;
-    lev[j] = (v >= 0 && v < kLevels) ? v : (int8_t)-1;
+    int8_t u = (v >= -1 && v < kLevels) ? v : (int8_t)-1;
+    if (a.causal && j < a.Nk) {
+      if (j * a.kv_blk > q_hi) u = -1;                                        // future block
+      else if (u > 0 && min((j + 1) * a.kv_blk, a.N) - 1 >= q_lo) u = 0;   // straddles
+    }
+    changed |= j < a.Nk && u != v;
+    lev[j] = u;
   }
+  if (__any_sync(0xffffffffu, changed) && lane == 0) atomicOr(err, kErrLevelMap);
   __syncwarp();
   emit_list_warp(lev, a.Nk, list + (long long)row * a.Nk, counts + row);
 }
@@ -710,7 +726,8 @@ cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int
   if (e != cudaSuccess) return e;
   const int nrows = p.B * p.Hq * L.Nq;
   map_to_list_kernel<<<(nrows + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, smem, st>>>(
-      a, rows_per_cta, nrows, map, (int*)(ws + L.list), (int4*)(ws + L.counts));
+      a, rows_per_cta, nrows, map, (int*)(ws + L.list), (int4*)(ws + L.counts),
+      (int*)(ws + L.err));
   return cudaGetLastError();
 }
 

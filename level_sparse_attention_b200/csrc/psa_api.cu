@@ -205,7 +205,7 @@ psa_status_t psa_check_device(const psa_params_t* params, void* workspace, size_
   if (host_err != 0) {
     if (cudaMemsetAsync(dev_err, 0, sizeof(int), st) != cudaSuccess) return PSA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return PSA_ERR_CUDA;
-    return PSA_ERR_DEVICE_TIMEOUT;
+    return (host_err & kErrTimeout) ? PSA_ERR_DEVICE_TIMEOUT : PSA_ERR_LEVEL_MAP;
   }
   return PSA_OK;
 }
@@ -219,6 +219,9 @@ const char* psa_status_string(psa_status_t status) {
     case PSA_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than psa_workspace_size()";
     case PSA_ERR_CUDA: return "CUDA error";
     case PSA_ERR_DEVICE_TIMEOUT: return "a kernel gave up waiting on the device (timeout)";
+    case PSA_ERR_LEVEL_MAP: return "a caller's level map broke the contract and was corrected "
+                                   "(values outside -1..3 pruned; causal: future blocks pruned, "
+                                   "diagonal blocks at level 0)";
   }
   return "unknown status";
 }

@@ -13,7 +13,8 @@ namespace psa {
 
 constexpr int kLevels = 4;
 constexpr int kMaxNk = 8192;          // KV blocks per query block row (N <= 524288 at 64)
-constexpr int kErrTimeout = 1;        // bit in the device error word
+constexpr int kErrTimeout = 1;        // bits in the device error word: a wait ran out,
+constexpr int kErrLevelMap = 2;       // a caller's level map was corrected
 
 inline __host__ __device__ size_t cdiv(size_t a, size_t b) { return (a + b - 1) / b; }
 inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -18,9 +18,12 @@ import workloads as W
 BF16_MAX_ABS, BF16_MEAN_REL = 2e-2, 5e-3
 F32_MAX_ABS = 1e-4
 # Map parity: a level may differ only when the oracle's cumulative mass is this
-# close to a threshold separating the two levels, or the block's mass is this
-# close to that of a block holding the GPU's level (a near-tie in the ranking).
-MAP_EPS_C, MAP_EPS_P = 1e-5, 1e-6
+# close to a threshold separating the two levels (absolute), or the block's
+# mass is this close, relative to the larger of the two, to that of a block
+# holding the GPU's level (a near-tie in the ranking).  The GPU's block masses
+# carry a relative error of about 1e-5 (split-precision fp32 logits, fp32
+# softmax), so two masses closer than that may rank either way.
+MAP_EPS_C, MAP_EPS_P_REL = 1e-5, 1e-4
 
 
 def to_device(x: np.ndarray, dtype: str) -> torch.Tensor:
@@ -113,7 +116,7 @@ def map_mismatch_report(gpu_map: np.ndarray, mask: O.MaskResult, tau: Sequence[f
             near_thr += 1
             continue
         pj = mask.mass[a, j]
-        close = np.abs(mask.mass[a] - pj) <= MAP_EPS_P
+        close = np.abs(mask.mass[a] - pj) <= MAP_EPS_P_REL * np.maximum(mask.mass[a], pj)
         close[j] = False
         if np.any(close & (om[a] == g)):
             near_tie += 1

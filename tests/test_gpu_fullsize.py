@@ -17,9 +17,26 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 FULL = ["wan2.1_1.3b", "cogvideox_5b", "wan2.1_14b_720p", "qwen2.5_vl_7b"]
 
 
+# Mismatches excused as near-threshold or near-tie may be at most this
+# fraction of the sampled heads' map entries.
+EXEMPT_BOUND = 1e-3
+SMS = 148                                  # persistent CTAs of the attention kernel
+
+
 def sample_heads(w):
     hs = sorted({0, w.Hq // 2, w.Hq - 1})
     return [(0, h) for h in hs]
+
+
+def sample_blocks(w, h, rng, n=16):
+    """At least n query blocks of head h: the first and last, the first and
+    last of every band of the persistent grid (items (b*Hq + h)*Nq + a, taken
+    SMS at a time), and random ones."""
+    edge = [a for a in range(w.Nq) if (h * w.Nq + a) % SMS in (0, SMS - 1)]
+    blocks = {0, w.Nq - 1} | set(edge)
+    while len(blocks) < n:
+        blocks.add(int(rng.integers(0, w.Nq)))
+    return sorted(blocks)
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -31,7 +48,7 @@ def test_full_size_sampled(name):
     gm = run.level_map.cpu().numpy()
     grp = w.Hq // w.Hkv
     rng = np.random.default_rng(7)
-    total_thr = total_tie = 0
+    total_thr = total_tie = entries = 0
     for b, h in sample_heads(w):
         Q = inp.as_f64("q", b, h)
         K, V = inp.as_f64("k", b, h // grp), inp.as_f64("v", b, h // grp)
@@ -43,8 +60,9 @@ def test_full_size_sampled(name):
         assert unexplained == 0, (name, h, unexplained, thr, tie)
         total_thr += thr
         total_tie += tie
-        # output rows of a few query blocks (first, last, random), oracle on the GPU's map
-        blocks = sorted({0, w.Nq - 1, int(rng.integers(0, w.Nq))})
+        entries += gm[b, h].size
+        # output rows of sampled query blocks, oracle on the GPU's map
+        blocks = sample_blocks(w, h, rng)
         sub = np.full_like(gm[b, h], -1)
         sub[blocks] = gm[b, h][blocks]
         ref_O, ref_lse = O.pyramid_attention(Q, pyr, sub, w.q_blk, w.kv_blk, s, w.causal)
@@ -58,7 +76,9 @@ def test_full_size_sampled(name):
         for a in range(w.Nq):
             last = min((a + 1) * w.q_blk, w.N) - 1
             assert np.all(gm[:, :, a, last // w.kv_blk + 1:] == -1)
-    print(f"{name}: near-threshold {total_thr}, near-tie {total_tie} exempt mismatches")
+    print(f"{name}: near-threshold {total_thr}, near-tie {total_tie} exempt mismatches "
+          f"of {entries} sampled map entries")
+    assert total_thr + total_tie <= EXEMPT_BOUND * entries, (total_thr, total_tie, entries)
 
 
 def test_max_size_single_head():

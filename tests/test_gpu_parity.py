@@ -62,6 +62,20 @@ CASES = {
                                            grid=(1, 47, 203), coarse=(1, 12, 51),
                                            forced_prefix_tokens=0, seed=22, target="alpha:1.0",
                                            assign="quantile"),
+    # binary keep/drop (tau_0 = ... = tau_3: every kept block at level 0, the
+    # baseline the method generalises), 150 blocks per row through the
+    # candidate cut (small tau)
+    "bf16_binary_cut": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0,
+                                        grid=(1, 47, 203), coarse=(1, 12, 51),
+                                        forced_prefix_tokens=0, seed=24, target="binary:0.15"),
+    # binary keep/drop, causal with grouped queries, through the candidate cut
+    "bf16_binary_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 47, 203),
+                                           coarse=(1, 12, 51), seed=25, target="binary:0.3"),
+    # binary keep/drop with tau = 1: every visible block kept at level 0 (dense
+    # attention), the full sort of every row
+    "bf16_binary_full": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, n_text=0,
+                                         grid=(1, 47, 203), coarse=(1, 12, 51),
+                                         forced_prefix_tokens=0, seed=26, target="binary:1.0"),
 }
 
 _cache = {}
@@ -232,6 +246,85 @@ def test_quantile_long_rows_shared_memory_sort():
     # every row keeps exactly K_3 blocks
     K3 = O.quotas(w.Nk, W.thresholds(w))[3]
     assert np.all((gm >= 0).sum(-1) == K3)
+
+
+@pytest.mark.parametrize("assign", ["threshold", "quantile"])
+@pytest.mark.parametrize("tau", [0.05, 1.0])
+def test_long_rows_binary_and_quantile_shared_memory_path(assign, tau):
+    """Rows of more than 1024 KV blocks (one head, N = 66000: 1032 blocks per
+    row) sort in shared memory; binary keep/drop (tau_0 = ... = tau_3) through
+    the candidate cut (tau = 0.05) and the full sort (tau = 1), under both
+    rules.  The map against the oracle's."""
+    w = W.with_overrides(BASE["cogvideox_5b"], Hq=1, Hkv=1, n_text=0, grid=(4, 110, 150),
+                         coarse=(1, 28, 38), forced_prefix_tokens=0, seed=27,
+                         target=f"binary:{tau}", assign=assign)
+    assert w.Nk == 1032
+    inp = W.make_inputs(w)
+    run = G.run_stages(w, inp)
+    gm = run.level_map.cpu().numpy()[0, 0]
+    Q, K = inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0)
+    pyr = O.build_pyramid(K, K)
+    z = O.block_logits(O.query_block_means(Q, w.q_blk), pyr, w.kv_blk, 1.0 / np.sqrt(w.d))
+    tau4 = W.thresholds(w)
+    mask = O.assign_levels(z, tau4, w.N, w.q_blk, w.kv_blk, w.causal, 0, assign)
+    assert G.map_mismatch_report(gm, mask, tau4, assign)[0] == 0
+    assert set(np.unique(gm).tolist()) <= {-1, 0}
+    if tau == 1.0:
+        assert np.all(gm == 0)
+
+
+@pytest.mark.parametrize("name", ["bf16_gqa_causal", "bf16_q64_causal"])
+def test_causal_caller_map_is_corrected(name):
+    """A caller's causal map that breaks the contract: future blocks at level 2,
+    diagonal blocks at level 3, a value of 7 and one of -5.  The kernels attend
+    to the corrected map (future blocks pruned, diagonal blocks at level 0,
+    out-of-range values pruned), equal to the oracle's, and the error word
+    reports the correction as PSA_ERR_LEVEL_MAP, which the check clears."""
+    w, inp, _, _ = setup(name)
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    m = rng.integers(-1, 4, size=(w.B, w.Hq, w.Nq, w.Nk)).astype(np.int8)
+    m[..., -1] = 2                            # the future of every query block but the last
+    for a in range(w.Nq):                     # diagonal blocks at a pooled level
+        for j in range(w.Nk):
+            if O.straddles(a, j, w.N, w.q_blk, w.kv_blk):
+                m[:, :, a, j] = 3
+    m[0, 0, 1, 0], m[0, w.Hq - 1, 2, 1] = 7, -5
+    p = G.params_for(w)
+    ws = P.new_workspace(p)
+    q, k, v = (G.to_device(x, w.dtype) for x in (inp.q, inp.k, inp.v))
+    out = torch.zeros_like(q)
+    lse = torch.zeros((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    P.build_pyramid(p, k, v, ws)
+    P.attention_fwd(p, q, k, v, ws, out, lse, torch.from_numpy(m).cuda())
+    torch.cuda.synchronize()
+    with pytest.raises(P.PSAError) as e:
+        P.check_device(p, ws)
+    assert e.value.status == 7
+    P.check_device(p, ws)                     # cleared
+    fixed = np.stack([np.stack([O.correct_map(m[b, h], w.N, w.q_blk, w.kv_blk, True)[0]
+                                for h in range(w.Hq)]) for b in range(w.B)])
+    assert int((fixed != m).sum()) > 0
+    # the list the kernel built is the corrected map's
+    counts = run_view(ws, p, "counts", (w.B, w.Hq, w.Nq, 4), torch.int32)
+    lst = run_view(ws, p, "list", (w.B, w.Hq, w.Nq, w.Nk), torch.int32)
+    for h in range(w.Hq):
+        for a in range(w.Nq):
+            want = [j for l in range(4) for j in range(w.Nk) if fixed[0, h, a, j] == l]
+            assert counts[0, h, a].tolist() == [int((fixed[0, h, a] == l).sum()) for l in range(4)]
+            assert lst[0, h, a, :len(want)].tolist() == want
+    ref = G.oracle_heads(w, inp, [(0, h) for h in range(w.Hq)], level_map=m)
+    gO, glse = G.to_f64(out), lse.cpu().numpy().astype(np.float64)
+    for (b, h), r in ref.items():
+        G.compare_out(gO[b, h], r.O, w.dtype)
+        G.compare_lse(glse[b, h], r.lse, w.dtype)
+    # a map that keeps the contract is not flagged
+    P.attention_fwd(p, q, k, v, ws, out, lse, torch.from_numpy(fixed).cuda())
+    torch.cuda.synchronize()
+    P.check_device(p, ws)
+
+
+def run_view(ws, p, key, shape, dtype):
+    return P.workspace_view(ws, P.workspace_layout(p)[key], shape, dtype).cpu().numpy()
 
 
 def test_no_device_timeouts_recorded():

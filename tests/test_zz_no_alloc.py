@@ -13,7 +13,6 @@ first failure has already run every other test.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -65,9 +64,8 @@ def test_noalloc_matches_psa_forward_twice_in_a_row():
         P.forward(p, q, k, v, o_ref, ws, lse_ref, lm_ref)
         assert _call(p, q, k, v, o_na, lse_na, lm_na) == 0
         torch.cuda.synchronize()
+        # the same kernels on the same inputs: identical bits, so a region of
+        # the shared array that a call failed to rewrite would show
         assert torch.equal(lm_na, lm_ref)
-        a, b = G.to_f64(o_na), G.to_f64(o_ref)
-        for h in range(w.Hq):
-            G.compare_out(a[0, h], b[0, h], w.dtype)
-            G.compare_lse(lse_na[0, h].cpu().numpy().astype(np.float64),
-                          lse_ref[0, h].cpu().numpy().astype(np.float64), w.dtype)
+        assert torch.equal(o_na, o_ref)
+        assert torch.equal(lse_na, lse_ref)

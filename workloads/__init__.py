@@ -56,7 +56,8 @@ class Workload:
     causal: bool
     forced_prefix_tokens: int       # KV blocks holding any of these tokens get level 0
     seed: int
-    target: str                     # how tau is chosen: "fixed", "alpha:0.15", "skip:0.91", "keep:0.35"
+    target: str                     # how tau is chosen: "fixed", "alpha:0.15", "binary:0.2",
+                                    # "skip:0.91", "keep:0.35"
     pool: Tuple[int, int, int, int] = (1, 2, 4, 8)
     assign: str = "threshold"       # level assignment rule: "threshold" or "quantile"
 
@@ -108,11 +109,15 @@ BY_NAME = {w.name: w for w in WORKLOADS}
 def thresholds(w: Workload) -> Tuple[float, float, float, float]:
     """The cumulative-mass thresholds tau_0..tau_3 of a workload.
 
-    The tiny case fixes them; "alpha:X" scales the shape to tau_3 = X; the
-    others read the alpha frozen in ``thresholds.json`` (written by
+    The tiny case fixes them; "alpha:X" scales the shape to tau_3 = X;
+    "binary:X" sets all four to X (keep/drop: every kept block at level 0);
+    the others read the alpha frozen in ``thresholds.json`` (written by
     ``oracle/tune_thresholds.py``)."""
     if w.target == "fixed":
         return TAU_SHAPE
+    if w.target.startswith("binary:"):
+        x = float(w.target.split(":", 1)[1])
+        return (x, x, x, x)
     if w.target.startswith("alpha:"):
         alpha = float(w.target.split(":", 1)[1])
         return tuple(float(alpha * t / TAU_SHAPE[-1]) for t in TAU_SHAPE)
