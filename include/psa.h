@@ -47,7 +47,8 @@ typedef enum {
   PSA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < psa_workspace_size(params)    */
   PSA_ERR_CUDA = 5,                 /* a CUDA call or launch failed                    */
   PSA_ERR_DEVICE_TIMEOUT = 6,       /* a kernel gave up waiting (see psa_check_device) */
-  PSA_ERR_LEVEL_MAP = 7             /* a caller's level map was corrected (see psa_attention_fwd) */
+  PSA_ERR_LEVEL_MAP = 7,            /* a caller's level map was corrected (see psa_attention_fwd) */
+  PSA_ERR_DEVICE_BOUNDS = 8         /* debug builds: a work list failed its bounds check         */
 } psa_status_t;
 
 typedef enum { PSA_F32 = 0, PSA_BF16 = 1 } psa_dtype_t;
@@ -272,7 +273,8 @@ psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void*
 
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns PSA_ERR_DEVICE_TIMEOUT if a kernel gave up waiting since the last
- * check, else PSA_ERR_LEVEL_MAP if a caller's level map was corrected
+ * check, else PSA_ERR_DEVICE_BOUNDS if (debug builds) a work list failed its
+ * bounds check, else PSA_ERR_LEVEL_MAP if a caller's level map was corrected
  * (psa_attention_fwd, psa_backward), PSA_ERR_CUDA if the stream reported an
  * error, else PSA_OK. */
 psa_status_t psa_check_device(const psa_params_t* params, void* workspace,
@@ -291,6 +293,17 @@ psa_status_t psa_check_device(const psa_params_t* params, void* workspace,
  * argument or a limit outside 1 ns .. 1 s, PSA_ERR_CUDA for a launch error. */
 psa_status_t psa_selftest_wait_timeout(const psa_params_t* params, void* workspace,
                                        size_t workspace_bytes, uint64_t limit_ns, void* stream);
+
+/* 1 when the library was compiled with PSA_DEBUG (libpsa_debug.so), else 0;
+ * the method has no counterpart.  A debug build checks, on the device, every
+ * work list in the workspace before the attention kernels (forward and
+ * backward) walk it: a query block whose level counts are negative or add up
+ * to more than ceil(N / kv_blk), or whose entries leave that range or are not
+ * increasing inside a level, is skipped (O = 0, lse = -inf, no gradient) and
+ * recorded in the error word, which psa_check_device reports as
+ * PSA_ERR_DEVICE_BOUNDS.  Lists written by this library always pass; the
+ * check guards against a workspace corrupted between calls.  Nothing traps. */
+int psa_debug_build(void);
 
 /* Static description of a status code. */
 const char* psa_status_string(psa_status_t status);

@@ -17,11 +17,13 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpsa.so")
+# the same library compiled with PSA_DEBUG (device-side work-list bounds checks)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libpsa_debug.so")
 
 F32, BF16 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "misaligned",
            4: "workspace too small", 5: "CUDA error", 6: "device timeout",
-           7: "level map corrected"}
+           7: "level map corrected", 8: "work list out of bounds (debug build)"}
 
 
 class PSAError(RuntimeError):
@@ -42,6 +44,7 @@ class Params(ctypes.Structure):
 
 
 _lib = None
+_debug_lib = None
 
 
 def lib() -> ctypes.CDLL:
@@ -49,9 +52,24 @@ def lib() -> ctypes.CDLL:
     There is no fallback: a missing library is an error."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing; run python -m level_sparse_attention_b200.build")
-        L = ctypes.CDLL(LIB_PATH)
+        _lib = _load(LIB_PATH)
+    return _lib
+
+
+def debug_lib() -> ctypes.CDLL:
+    """Load libpsa_debug.so, the PSA_DEBUG build of the same sources (built by
+    ``python -m level_sparse_attention_b200.build --debug``)."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+    return _debug_lib
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if True:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; run python -m level_sparse_attention_b200.build")
+        L = ctypes.CDLL(path)
         P, vp, sz = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_size_t
         sigs = {
             "psa_workspace_size": (sz, [P]),
@@ -66,20 +84,20 @@ def lib() -> ctypes.CDLL:
             "psa_forward_host": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                 ctypes.c_int, vp, vp, vp]),
             "psa_backward_workspace_size": (sz, [P]),
+            "psa_debug_build": (ctypes.c_int, []),
             "psa_backward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp, vp,
                                             vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
             fn.restype, fn.argtypes = res, args
-        _lib = L
-    return _lib
+    return L
 
 
 EXPORTED = ("psa_workspace_size", "psa_build_pyramid", "psa_score_and_mask",
             "psa_attention_fwd", "psa_forward", "psa_check_device", "psa_status_string",
             "psa_forward_noalloc", "psa_selftest_wait_timeout", "psa_forward_host",
-            "psa_backward_workspace_size", "psa_backward")
+            "psa_backward_workspace_size", "psa_backward", "psa_debug_build")
 
 
 def status_string(status: int) -> str:

@@ -662,6 +662,38 @@ __global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
   emit_list_warp(lev, a.Nk, list + (long long)row * a.Nk, counts + row);
 }
 
+#ifdef PSA_DEBUG
+// Debug builds only: every consumer of a work list reads entries by index and
+// turns them into addresses, so a list that no kernel of this library wrote
+// (a corrupted workspace) is checked first.  A row whose counts are negative
+// or add up to more than Nk, or whose entries leave [0, Nk) or are not
+// increasing inside a level, is reported in the error word (kErrListBounds)
+// and emptied (its counts set to 0), so that no kernel reads through it.
+__global__ void list_check_kernel(MaskArgs a, int nrows, const int* __restrict__ list,
+                                  int4* __restrict__ counts, int* __restrict__ err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= nrows) return;
+  const int4 c = counts[row];
+  const long long tot = (long long)c.x + c.y + c.z + c.w;
+  bool bad = c.x < 0 || c.y < 0 || c.z < 0 || c.w < 0 || tot > a.Nk;
+  if (!bad) {
+    const int* lrow = list + (long long)row * a.Nk;
+    const int f1 = c.x, f2 = f1 + c.y, f3 = f2 + c.z;
+    for (int e = lane; e < (int)tot; e += 32) {
+      const int j = lrow[e];
+      const bool first = e == 0 || e == f1 || e == f2 || e == f3;
+      bad |= j < 0 || j >= a.Nk || (!first && j <= lrow[e - 1]);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+  }
+  if (bad && lane == 0) {
+    counts[row] = make_int4(0, 0, 0, 0);
+    atomicOr(err, kErrListBounds);
+  }
+}
+#endif
+
 int next_pow2(int x) {
   int n = 1;
   while (n < x) n <<= 1;
@@ -714,6 +746,19 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
     case 1024: return go(assign_kernel<32>);
     default: return go(assign_kernel<0>);
   }
+}
+
+cudaError_t launch_list_check(const psa_params_t& p, const Layout& L, char* ws, cudaStream_t st) {
+#ifdef PSA_DEBUG
+  const MaskArgs a = make_mask_args(p, L, 0.f);
+  const int nrows = p.B * p.Hq * L.Nq;
+  list_check_kernel<<<(nrows + 7) / 8, 256, 0, st>>>(a, nrows, (const int*)(ws + L.list),
+                                                     (int4*)(ws + L.counts), (int*)(ws + L.err));
+  return cudaGetLastError();
+#else
+  (void)p; (void)L; (void)ws; (void)st;
+  return cudaSuccess;
+#endif
 }
 
 cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int8_t* map,

@@ -87,6 +87,7 @@ psa_status_t run_attention(const psa_params_t* p, const Layout& L, const void* Q
     psa_status_t r = from_cuda(launch_map_to_list(*p, L, map, (char*)ws, st));
     if (r != PSA_OK) return r;
   }
+  if (psa_status_t r = from_cuda(launch_list_check(*p, L, (char*)ws, st)); r != PSA_OK) return r;
   if (attention_tc_supported(*p))
     return from_cuda(launch_attention_tc(*p, L, s, Q, K, V, (char*)ws, O, lse, st));
   return from_cuda(launch_attention_simt(*p, L, s, Q, K, V, (const char*)ws, O, lse, st));
@@ -183,6 +184,7 @@ psa_status_t psa_backward(const psa_params_t* params, const void* Q, const void*
   if ((r = run_pyramid(params, L, K, V, workspace, st)) != PSA_OK) return r;
   if (level_map && (r = from_cuda(launch_map_to_list(*params, L, level_map, (char*)workspace, st))) != PSA_OK)
     return r;
+  if ((r = from_cuda(launch_list_check(*params, L, (char*)workspace, st))) != PSA_OK) return r;
   if ((r = from_cuda(launch_bwd_prep(*params, B, a, st))) != PSA_OK) return r;
   r = from_cuda(attention_bwd_tc_supported(*params) ? launch_attention_bwd_tc(*params, L, B, a, st)
                                                     : launch_attention_bwd_simt(*params, L, B, a, st));
@@ -205,9 +207,18 @@ psa_status_t psa_check_device(const psa_params_t* params, void* workspace, size_
   if (host_err != 0) {
     if (cudaMemsetAsync(dev_err, 0, sizeof(int), st) != cudaSuccess) return PSA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return PSA_ERR_CUDA;
-    return (host_err & kErrTimeout) ? PSA_ERR_DEVICE_TIMEOUT : PSA_ERR_LEVEL_MAP;
+    if (host_err & kErrTimeout) return PSA_ERR_DEVICE_TIMEOUT;
+    return (host_err & kErrListBounds) ? PSA_ERR_DEVICE_BOUNDS : PSA_ERR_LEVEL_MAP;
   }
   return PSA_OK;
+}
+
+int psa_debug_build(void) {
+#ifdef PSA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 const char* psa_status_string(psa_status_t status) {
@@ -219,6 +230,8 @@ const char* psa_status_string(psa_status_t status) {
     case PSA_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than psa_workspace_size()";
     case PSA_ERR_CUDA: return "CUDA error";
     case PSA_ERR_DEVICE_TIMEOUT: return "a kernel gave up waiting on the device (timeout)";
+    case PSA_ERR_DEVICE_BOUNDS: return "a work list in the workspace failed the debug build's "
+                                       "bounds check (its query block was skipped)";
     case PSA_ERR_LEVEL_MAP: return "a caller's level map broke the contract and was corrected "
                                    "(values outside -1..3 pruned; causal: future blocks pruned, "
                                    "diagonal blocks at level 0)";

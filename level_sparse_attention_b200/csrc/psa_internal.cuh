@@ -14,7 +14,8 @@ namespace psa {
 constexpr int kLevels = 4;
 constexpr int kMaxNk = 8192;          // KV blocks per query block row (N <= 524288 at 64)
 constexpr int kErrTimeout = 1;        // bits in the device error word: a wait ran out,
-constexpr int kErrLevelMap = 2;       // a caller's level map was corrected
+constexpr int kErrLevelMap = 2;       // a caller's level map was corrected,
+constexpr int kErrListBounds = 4;     // (debug builds) a work list failed its bounds check
 
 inline __host__ __device__ size_t cdiv(size_t a, size_t b) { return (a + b - 1) / b; }
 inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -128,6 +129,9 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
                           int8_t* user_map, float* block_mass, cudaStream_t st);
 cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int8_t* map,
                                char* ws, cudaStream_t st);
+// Debug builds (PSA_DEBUG): checks every work list before it is walked; a
+// no-op otherwise.
+cudaError_t launch_list_check(const psa_params_t& p, const Layout& L, char* ws, cudaStream_t st);
 cudaError_t launch_attention_simt(const psa_params_t& p, const Layout& L, float scale,
                                   const void* Q, const void* K, const void* V, const char* ws,
                                   void* O, float* lse, cudaStream_t st);

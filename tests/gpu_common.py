@@ -81,6 +81,19 @@ def run_stages(w: W.Workload, inp: W.Inputs, tau=None, external_map: Optional[np
             ext = torch.from_numpy(np.ascontiguousarray(external_map, dtype=np.int8)).cuda()
         P.attention_fwd(p, q, k, v, ws, out, lse, ext)
     torch.cuda.synchronize()
+    # a caller's map that breaks the contract (out-of-range values; causally,
+    # future or pooled diagonal blocks) is corrected on the device and
+    # reported as PSA_ERR_LEVEL_MAP; the oracle corrects it the same way
+    changed = 0
+    if external_map is not None and not fused:
+        changed = sum(O.correct_map(external_map[b, h], w.N, w.q_blk, w.kv_blk, w.causal)[1]
+                      for b in range(w.B) for h in range(w.Hq))
+    if changed:
+        try:
+            P.check_device(p, ws)
+            raise AssertionError("a corrected map was not reported")
+        except P.PSAError as e:
+            assert e.status == 7, e
     P.check_device(p, ws)
     return GpuRun(p, ws, q, k, v, lm, mass, out, lse)
 

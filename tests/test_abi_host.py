@@ -26,6 +26,17 @@ def test_library_exports_every_declared_entry_point():
         assert hasattr(L, n), n
 
 
+def test_debug_library_exports_the_same_entry_points():
+    """libpsa_debug.so (PSA_DEBUG: device-side work-list bounds checks) is the
+    same ABI; psa_debug_build tells the two apart."""
+    D = P.debug_lib()
+    for n in header_functions():
+        assert hasattr(D, n), n
+    assert D.psa_debug_build() == 1
+    assert P.lib().psa_debug_build() == 0
+    assert P.status_string(8).startswith("a work list")
+
+
 def test_workspace_layout_matches_library():
     for w in [(1, 12, 12, 32760, 128, 128, torch.bfloat16), (1, 2, 2, 1024, 64, 64, torch.float32),
               (2, 28, 4, 16384, 128, 128, torch.bfloat16), (1, 3, 1, 77, 64, 128, torch.bfloat16)]:
