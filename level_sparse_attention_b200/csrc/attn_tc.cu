@@ -58,15 +58,7 @@ constexpr int kSoftWarp0 = 4;            // first softmax warp (warpgroup aligne
 constexpr int kThreads = 128 + 128 * kStreams;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-#ifndef PSA_RESCALE_LOG2
-#define PSA_RESCALE_LOG2 8.0f
-#endif
-#ifndef PSA_EXP_BF16X2
-#define PSA_EXP_BF16X2 0
-#endif
-constexpr float kRescaleLog2 = PSA_RESCALE_LOG2;   // lazy rescale threshold (log2 of the factor)
-// exponentials of the softmax as packed bf16 pairs on the transcendental unit
-constexpr bool kExpBf16x2 = PSA_EXP_BF16X2 != 0;
+constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
 
 template <int D>
 struct Cfg {
@@ -152,19 +144,6 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
   f2unpack(T, t0, t1);
   y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// 2^x of a bf16 pair (one transcendental-unit operation for both halves)
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-// {lo, hi} rounded to a bf16 pair, lo in the low half
-__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
 }
 
 // How many of every 8 exponential pairs of a softmax tile take the FMA-pipe
@@ -586,16 +565,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < 64; c += 2) {
             float d0, d1, p0, p1;
             f2unpack(fadd2(f2pack(x[c], x[c + 1]), nm2), d0, d1);
-            if constexpr (kExpBf16x2) {
-              // the pair rounded to bf16, both exponentials in one operation;
-              // the row sum takes the bf16 values the PV product uses
-              const uint32_t e = ex2_bf16x2(cvt_bf16x2(d0, d1));
-              pk[c / 2] = e;
-              const uint64_t pp = f2pack(__uint_as_float(e << 16), __uint_as_float(e & 0xffff0000u));
-              if ((c >> 1) & 1) acc1 = fadd2(acc1, pp);
-              else acc0 = fadd2(acc0, pp);
-              continue;
-            }
             if (((c >> 1) & 7) < kPolyPairs) {
               exp2_poly2(d0, d1, p0, p1);
             } else {
