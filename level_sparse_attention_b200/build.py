@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = ["pyramid.cu", "mask.cu", "score_tc.cu", "attn_simt.cu", "attn_tc.cu", "psa_api.cu",
            "psa_noalloc.cu", "psa_selftest.cu", "psa_host.cu", "bwd_aux.cu", "attn_bwd_simt.cu",
-           "attn_bwd_tc.cu", "similarity.cu"]
+           "attn_bwd_tc.cu"]
 LIB = os.path.join(HERE, "libpsa.so")
 DEBUG_LIB = os.path.join(HERE, "libpsa_debug.so")
 

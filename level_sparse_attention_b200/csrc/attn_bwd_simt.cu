@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(512) attn_bwd_simt_kernel(BwdSimtArgs a, const
   float* Vs = Ks + kTileKeys * D;                  // [kTileKeys][D]
   float* Ps = Vs + kTileKeys * D;                  // [q_blk][kTileKeys]
   float* Xs = Ps + a.q_blk * kTileKeys;            // [q_blk][kTileKeys]  dX
+  pdl_wait();
   float* bias = Xs + a.q_blk * kTileKeys;          // [kTileKeys] log2 c, -inf = no key
   int* kpos = reinterpret_cast<int*>(bias + kTileKeys);   // token position or INT_MIN
   int* dst = kpos + kTileKeys;                     // (level << 24) | pooled row, or -1
@@ -204,10 +205,9 @@ cudaError_t launch_bwd_simt_typed(const BwdSimtArgs& a, int grid, const Layout& 
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_simt_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_simt_kernel<T, D><<<grid, threads, smem, st>>>(
-      a, (const T*)x.Q, (const T*)x.dO, (const int*)(x.ws + L.list),
-      (const int4*)(x.ws + L.counts), (T*)x.dQ);
-  return cudaGetLastError();
+  return launch_dependent(attn_bwd_simt_kernel<T, D>, dim3(grid), dim3(threads), smem, st, a,
+                          (const T*)x.Q, (const T*)x.dO, (const int*)(x.ws + L.list),
+                          (const int4*)(x.ws + L.counts), (T*)x.dQ);
 }
 
 }  // namespace

@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(512) attn_simt_kernel(SimtArgs a, const T* __r
   float* Vs = Ks + kTileKeys * D;      // [kTileKeys][D]
   float* bias = Vs + kTileKeys * D;    // [kTileKeys] log2 c, -inf = no key
   int* kpos = reinterpret_cast<int*>(bias + kTileKeys);   // [kTileKeys] token position or INT_MIN
+  pdl_wait();
 
   const int row = blockIdx.x;          // (b*Hq + hq) * Nq + qa
   const int qa = row % a.Nq;
@@ -186,9 +187,9 @@ cudaError_t launch_simt_typed(const SimtArgs& a, int q_blk, int grid, const void
   cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attn_simt_kernel<T, D><<<grid, threads, smem, st>>>(
-      a, (const T*)Q, (const int*)(ws + L.list), (const int4*)(ws + L.counts), (T*)O, lse);
-  return cudaGetLastError();
+  return launch_dependent(attn_simt_kernel<T, D>, dim3(grid), dim3(threads), smem, st, a,
+                          (const T*)Q, (const int*)(ws + L.list), (const int4*)(ws + L.counts),
+                          (T*)O, lse);
 }
 
 }  // namespace

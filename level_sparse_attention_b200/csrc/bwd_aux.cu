@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ O,
                                                        long long n_rows, float4* zero,
                                                        long long n_zero4) {
   constexpr int TPR = D / 8;
+  pdl_trigger();
+  pdl_wait();
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = gtid / TPR;
   const int part = (int)(gtid % TPR);
@@ -76,6 +78,8 @@ struct UnpoolArgs {
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_unpool_kernel(UnpoolArgs a, T* __restrict__ dK,
                                                          T* __restrict__ dV) {
+  pdl_trigger();
+  pdl_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n_items) return;
   constexpr int C4 = D / 4;
@@ -108,10 +112,9 @@ cudaError_t prep_typed(const psa_params_t& p, const BwdLayout& B, const BwdArgs&
   const long long blocks = (threads + 255) / 256;
   float4* zero = reinterpret_cast<float4*>(a.bws + B.acc_begin);
   const long long n_zero4 = (long long)((B.total - B.acc_begin) / 16);
-  bwd_prep_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
-      (const T*)a.O, (const T*)a.dO, reinterpret_cast<float*>(a.bws + B.delta), n_rows, zero,
-      n_zero4);
-  return cudaGetLastError();
+  return launch_dependent(bwd_prep_kernel<T, D>, dim3((unsigned)blocks), dim3(256), 0, st,
+                          (const T*)a.O, (const T*)a.dO, reinterpret_cast<float*>(a.bws + B.delta),
+                          n_rows, zero, n_zero4);
 }
 
 template <typename T, int D>
@@ -126,8 +129,8 @@ cudaError_t unpool_typed(const psa_params_t& p, const BwdLayout& B, const BwdArg
   u.N = p.N;
   u.n_items = (long long)p.B * p.Hkv * p.N * (D / 4);
   const long long blocks = (u.n_items + 255) / 256;
-  bwd_unpool_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(u, (T*)a.dK, (T*)a.dV);
-  return cudaGetLastError();
+  return launch_dependent(bwd_unpool_kernel<T, D>, dim3((unsigned)blocks), dim3(256), 0, st, u,
+                          (T*)a.dK, (T*)a.dV);
 }
 
 }  // namespace

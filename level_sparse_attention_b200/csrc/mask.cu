@@ -17,10 +17,11 @@
 //   qmean_kernel   one CTA per query block; streams Q once (HBM-bound).
 //   score_tc_kernel  split-precision tensor-core GEMM of query-block means
 //                  against the level-3 keys, logsumexp per KV block fused.
-//   assign_kernel  one warp per query block: softmax, bitonic sort of packed
-//                  (P, index) keys (in registers up to 1024 blocks, else in
-//                  shared memory), scan, cut, overrides, and the work list
-//                  (KV block indices grouped by level).
+//   assign_kernel  one warp per query block: softmax, a candidate cut (the
+//                  blocks above a bisected mass threshold, a prefix of the
+//                  ranking) sorted in registers, or a bitonic sort of the whole
+//                  row's packed (P, index) keys; scan, levels, overrides, and
+//                  the work list (KV block indices grouped by level).
 #include "psa_internal.cuh"
 
 namespace psa {
@@ -63,6 +64,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) qmean_kernel(MaskArgs a, const T* __restrict__ Q,
                                                     float* __restrict__ qmh,
                                                     float* __restrict__ qml) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;               // (b*Hq + h) * Nq + qa
   const int qa = row % a.Nq;
   const long long bh = row / a.Nq;
@@ -310,6 +313,8 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
                               int8_t* __restrict__ map_user, float* __restrict__ mass_user,
                               int* __restrict__ list, int4* __restrict__ counts) {
   extern __shared__ __align__(16) unsigned char smem[];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * rows_per_cta + warp;
   if (row >= nrows) return;                 // whole warp; no block barriers below
@@ -399,11 +404,10 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
           m = m_hi;
         } else {
           int m_lo = nvis;                 // the whole row: mass 1 >= target, nvis >= K_3
-          // once the candidates fit, a few more steps shrink them (ranking
-          // costs m per candidate, a step one pass over the row)
-          int extra = 0;
+          // stop as soon as the candidates fit (sorting them costs the same
+          // for any count up to kCand)
           for (int it = 0; it < 40; ++it) {
-            if (m_lo <= kCand && (m_lo <= 48 || extra++ >= 3)) break;
+            if (m_lo <= kCand) break;
             const float mid = 0.5f * (lo + hi);
             if (!(mid > lo && mid < hi)) break;
             int c;
@@ -430,35 +434,17 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
               key[pos++] = ((unsigned long long)__float_as_uint(pj[r]) << 32) | (0xffffffffu - (unsigned)i);
           }
           __syncwarp();
-          // a candidate's rank is the number of candidates with a larger key
-          // (P, then lower index), its running mass their total P
-          unsigned long long mk[kCandPerLane];
-          float c[kCandPerLane];
-          int rk[kCandPerLane];
+          // the candidates are a prefix of the ranking: sort them (P, then
+          // lower index, descending; zero keys pad to a power of two) and give
+          // each its level from its rank and the exclusive running mass
+          unsigned long long v[kCandPerLane];
 #pragma unroll
           for (int r = 0; r < kCandPerLane; ++r) {
-            const int i = lane + 32 * r;
-            mk[r] = i < m ? key[i] : ~0ull;
-            c[r] = 0.f;
-            rk[r] = 0;
+            const int i = lane * kCandPerLane + r;
+            v[r] = i < m ? key[i] : 0ull;
           }
-          for (int jj = 0; jj < m; ++jj) {
-            const unsigned long long kj = key[jj];          // same address in every lane
-            const float pj_ = __uint_as_float((unsigned)(kj >> 32));
-#pragma unroll
-            for (int r = 0; r < kCandPerLane; ++r) {
-              const bool before = kj > mk[r];
-              c[r] += before ? pj_ : 0.f;
-              rk[r] += before;
-            }
-          }
-#pragma unroll
-          for (int r = 0; r < kCandPerLane; ++r) {
-            if (lane + 32 * r < m) {
-              const int j = (int)(0xffffffffu - (unsigned)(mk[r] & 0xffffffffu));
-              lev[j] = rule.level(c[r], rk[r]);
-            }
-          }
+          warp_bitonic_desc<kCandPerLane>(v);
+          levels_from_sorted<kCandPerLane>(v, m, rule, lev);
           done = true;
         }
       }
@@ -515,9 +501,8 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
         m = m_hi;
       } else {
         int m_lo = nvis;
-        int extra = 0;
         for (int it = 0; it < 40; ++it) {
-          if (m_lo <= kCandS && (m_lo <= 48 || extra++ >= 6)) break;
+          if (m_lo <= kCandS) break;
           const float mid = 0.5f * (lo + hi);
           if (!(mid > lo && mid < hi)) break;
           int c;
@@ -543,33 +528,15 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
           base += __popc(bal);
         }
         __syncwarp();
-        unsigned long long mk[kCandPerLaneS];
-        float c[kCandPerLaneS];
-        int rk[kCandPerLaneS];
+        // sort the candidates in registers and scan, as in the register path
+        unsigned long long v[kCandPerLaneS];
 #pragma unroll
         for (int r = 0; r < kCandPerLaneS; ++r) {
-          const int i = lane + 32 * r;
-          mk[r] = i < m ? cand[i] : ~0ull;
-          c[r] = 0.f;
-          rk[r] = 0;
+          const int i = lane * kCandPerLaneS + r;
+          v[r] = i < m ? cand[i] : 0ull;
         }
-        for (int jj = 0; jj < m; ++jj) {
-          const unsigned long long kj = cand[jj];           // same address in every lane
-          const float pj_ = pk(kj);
-#pragma unroll
-          for (int r = 0; r < kCandPerLaneS; ++r) {
-            const bool before = kj > mk[r];
-            c[r] += before ? pj_ : 0.f;
-            rk[r] += before;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kCandPerLaneS; ++r) {
-          if (lane + 32 * r < m) {
-            const int j = (int)(0xffffffffu - (unsigned)(mk[r] & 0xffffffffu));
-            lev[j] = rule.level(c[r], rk[r]);
-          }
-        }
+        warp_bitonic_desc<kCandPerLaneS>(v);
+        levels_from_sorted<kCandPerLaneS>(v, m, rule, lev);
         done = true;
       }
     }
@@ -639,6 +606,8 @@ __global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
                                    const int8_t* __restrict__ map, int* __restrict__ list,
                                    int4* __restrict__ counts, int* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem[];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * rows_per_cta + warp;
   if (row >= nrows) return;
@@ -671,6 +640,8 @@ __global__ void map_to_list_kernel(MaskArgs a, int rows_per_cta, int nrows,
 // and emptied (its counts set to 0), so that no kernel reads through it.
 __global__ void list_check_kernel(MaskArgs a, int nrows, const int* __restrict__ list,
                                   int4* __restrict__ counts, int* __restrict__ err) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= nrows) return;
@@ -710,10 +681,10 @@ cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, 
   float* qh = (float*)(ws + L.qmh);
   float* ql = (float*)(ws + L.qml);
   if (p.dtype == PSA_BF16)
-    qmean_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(a, (const __nv_bfloat16*)Q, qh, ql);
-  else
-    qmean_kernel<float><<<grid, threads, 0, st>>>(a, (const float*)Q, qh, ql);
-  return cudaGetLastError();
+    return launch_dependent(qmean_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st, a,
+                            (const __nv_bfloat16*)Q, qh, ql);
+  return launch_dependent(qmean_kernel<float>, dim3(grid), dim3(threads), 0, st, a,
+                          (const float*)Q, qh, ql);
 }
 
 cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, char* ws,
@@ -731,11 +702,10 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
   auto go = [&](auto kern) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 32 * rows_per_cta, smem, st>>>(
-        a, n2, rows_per_cta, nrows, (const float*)(ws + L.zlog), (const int8_t*)(ws + L.maxlev),
-        (int8_t*)(ws + L.map), user_map,
-        block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), dim3(32 * rows_per_cta), smem, st, a, n2,
+                            rows_per_cta, nrows, (const float*)(ws + L.zlog),
+                            (const int8_t*)(ws + L.maxlev), (int8_t*)(ws + L.map), user_map,
+                            block_mass, (int*)(ws + L.list), (int4*)(ws + L.counts));
   };
   switch (n2) {   // keys per lane for the register sort; larger rows sort in shared memory
     case 32: return go(assign_kernel<1>);
@@ -752,9 +722,8 @@ cudaError_t launch_list_check(const psa_params_t& p, const Layout& L, char* ws, 
 #ifdef PSA_DEBUG
   const MaskArgs a = make_mask_args(p, L, 0.f);
   const int nrows = p.B * p.Hq * L.Nq;
-  list_check_kernel<<<(nrows + 7) / 8, 256, 0, st>>>(a, nrows, (const int*)(ws + L.list),
-                                                     (int4*)(ws + L.counts), (int*)(ws + L.err));
-  return cudaGetLastError();
+  return launch_dependent(list_check_kernel, dim3((nrows + 7) / 8), dim3(256), 0, st, a, nrows,
+                          (const int*)(ws + L.list), (int4*)(ws + L.counts), (int*)(ws + L.err));
 #else
   (void)p; (void)L; (void)ws; (void)st;
   return cudaSuccess;
@@ -770,10 +739,9 @@ cudaError_t launch_map_to_list(const psa_params_t& p, const Layout& L, const int
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nrows = p.B * p.Hq * L.Nq;
-  map_to_list_kernel<<<(nrows + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, smem, st>>>(
-      a, rows_per_cta, nrows, map, (int*)(ws + L.list), (int4*)(ws + L.counts),
-      (int*)(ws + L.err));
-  return cudaGetLastError();
+  return launch_dependent(map_to_list_kernel, dim3((nrows + rows_per_cta - 1) / rows_per_cta),
+                          dim3(32 * rows_per_cta), smem, st, a, rows_per_cta, nrows, map,
+                          (int*)(ws + L.list), (int4*)(ws + L.counts), (int*)(ws + L.err));
 }
 
 }  // namespace psa

@@ -64,10 +64,7 @@ psa_status_t check_ptrs(std::initializer_list<const void*> required) {
 
 psa_status_t run_pyramid(const psa_params_t* p, const Layout& L, const void* K, const void* V,
                          void* ws, cudaStream_t st) {
-  psa_status_t r = from_cuda(launch_pyramid(*p, L, K, V, (char*)ws, st));
-  if (r == PSA_OK && p->sim_threshold > -1.f)
-    r = from_cuda(launch_similarity(*p, L, K, (char*)ws, st));
-  return r;
+  return from_cuda(launch_pyramid(*p, L, K, V, (char*)ws, st));
 }
 
 psa_status_t run_mask(const psa_params_t* p, const Layout& L, const void* Q, void* ws,

@@ -107,20 +107,53 @@ __device__ __forceinline__ float tf32_head(float x) {
   return __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
+// Programmatic dependent launch.  The short kernels of the library (pyramid,
+// query means, block logits, assignment, list kernels, the backward's prep and
+// unpool) are launched so that they may be scheduled before the kernel ahead
+// of them on the stream has finished (launch_dependent below), and call
+// pdl_wait() before their first global-memory access: that returns once the
+// previous grid has completed and its writes are visible, so ordering is
+// exactly that of plain launches, while the launch itself, and a kernel's
+// set-up of shared memory, barriers and TMEM, overlap the previous kernel's
+// tail.  They call pdl_trigger() once started, so that the next kernel's CTAs
+// are scheduled as their own retire.  Outside such a launch both are no-ops.
+// The persistent attention kernels (forward and backward) are plain launches:
+// a grid-dependency wait in them measured slower.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
 
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 }  // namespace psa
 
 // Host-side launchers implemented in the kernel files.
 namespace psa {
+// The pyramid of K and V; with sim_threshold > -1 also each KV block's largest
+// level under the cosine constraint (same launch, from the same loads of K).
 cudaError_t launch_pyramid(const psa_params_t& p, const Layout& L, const void* K, const void* V,
                            char* ws, cudaStream_t st);
-cudaError_t launch_similarity(const psa_params_t& p, const Layout& L, const void* K, char* ws,
-                              cudaStream_t st);
 cudaError_t launch_qmean(const psa_params_t& p, const Layout& L, const void* Q, char* ws,
                          cudaStream_t st);
 cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, char* ws,

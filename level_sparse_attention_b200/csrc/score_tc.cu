@@ -170,6 +170,8 @@ __global__ void __launch_bounds__(kThr, 1) score_tc_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();                               // query means and level-3 keys are complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -368,17 +370,12 @@ cudaError_t launch_score(const psa_params_t& p, const Layout& L, float scale, ch
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = prm.n_items < sms ? prm.n_items : sms;   // persistent: one CTA per SM
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  auto go = [&](auto kern) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    score_tc_kernel<128><<<grid, kThr, kSmem, st>>>(prm);
-  } else {
-    e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    score_tc_kernel<64><<<grid, kThr, kSmem, st>>>(prm);
-  }
-  return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), dim3(kThr), kSmem, st, prm);
+  };
+  return p.d == 128 ? go(score_tc_kernel<128>) : go(score_tc_kernel<64>);
 }
 
 }  // namespace psa
