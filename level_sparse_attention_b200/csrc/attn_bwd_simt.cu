@@ -1,6 +1,6 @@
 // Gradient of pyramid attention on CUDA cores (fp32 FMA): the path for fp32
-// inputs and for 64-row query blocks, which the tensor-core kernel does not
-// take.  The gradient is the chain rule through the forward pass of adaptive
+// inputs (the tensor-core kernel takes bf16 with 64- and 128-row query
+// blocks).  The gradient is the chain rule through the forward pass of adaptive
 // pyramid attention (top168.com article on PSA, component three) with the
 // level map held fixed; see bwd_internal.cuh for the formulas.
 //

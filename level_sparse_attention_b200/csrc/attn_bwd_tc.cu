@@ -1,5 +1,6 @@
 // Gradient of pyramid attention on the 5th-generation tensor cores (tcgen05 +
-// TMEM + TMA), bf16 inputs, fp32 accumulation, 128-row query blocks, d in
+// TMEM + TMA), bf16 inputs, fp32 accumulation, 128-row query blocks (64-row
+// blocks as 128-row tiles whose rows 64-127 have P = dS = 0), d in
 // {64, 128}.
 //
 // Method: the chain rule through adaptive pyramid attention (top168.com
@@ -91,6 +92,7 @@ struct __align__(64) BwdTcParams {
   __nv_bfloat16* dQ;
   int* err;
   int Hq, Hkv, N, Nq, Nk, causal, n_rows;
+  int qb;                                   // query rows per block: 128, or 64 (rows 64-127 dead)
   float scale, scale_log2;
 };
 
@@ -219,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         if (lane == 0) {
           mbar_expect_tx(bar(B_QFULL), 2 * C::T_BYTES);
           for (int h = 0; h < C::HALVES; ++h) {
-            tma_load_3d(sbase + C::OFF_Q + h * C::HALF, &p.tq, bar(B_QFULL), h * 64, qa * kBM, bhq);
-            tma_load_3d(sbase + C::OFF_DO + h * C::HALF, &p.tdo, bar(B_QFULL), h * 64, qa * kBM, bhq);
+            tma_load_3d(sbase + C::OFF_Q + h * C::HALF, &p.tq, bar(B_QFULL), h * 64, qa * p.qb, bhq);
+            tma_load_3d(sbase + C::OFF_DO + h * C::HALF, &p.tdo, bar(B_QFULL), h * 64, qa * p.qb, bhq);
           }
         }
         ++iq;
@@ -384,8 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
       const int bhk = (bhq / p.Hq) * p.Hkv + (bhq % p.Hq) / (p.Hq / p.Hkv);
-      const int qpos = qa * kBM + r;
-      const bool valid = qpos < p.N;
+      const int qpos = qa * p.qb + r;
+      // rows past a 64-row query block are dead: P = dS = 0 (so they add
+      // nothing to dK, dV), no dQ store
+      const bool valid = r < p.qb && qpos < p.N;
       const long long qrow = (long long)bhq * p.N + qpos;
       const float lse2 = valid && T > 0 ? p.lse[qrow] * kLog2e : -INFINITY;
       const float Di = valid && T > 0 ? p.delta[qrow] : 0.f;
@@ -589,7 +593,8 @@ cudaError_t launch_typed(const BwdTcParams& prm, cudaStream_t st) {
 }  // namespace
 
 bool attention_bwd_tc_supported(const psa_params_t& p) {
-  return p.dtype == PSA_BF16 && p.q_blk == 128 && p.kv_blk == 64 && (p.d == 64 || p.d == 128);
+  return p.dtype == PSA_BF16 && (p.q_blk == 128 || p.q_blk == 64) && p.kv_blk == 64 &&
+         (p.d == 64 || p.d == 128);
 }
 
 cudaError_t launch_attention_bwd_tc(const psa_params_t& p, const Layout& L, const BwdLayout& B,
@@ -620,6 +625,7 @@ cudaError_t launch_attention_bwd_tc(const psa_params_t& p, const Layout& L, cons
   prm.Hq = p.Hq; prm.Hkv = p.Hkv; prm.N = p.N; prm.Nq = L.Nq; prm.Nk = L.Nk;
   prm.causal = p.causal;
   prm.n_rows = BHq * L.Nq;
+  prm.qb = p.q_blk;
   prm.scale = a.scale;
   prm.scale_log2 = a.scale * kLog2e;
   return p.d == 128 ? launch_typed<128>(prm, st) : launch_typed<64>(prm, st);

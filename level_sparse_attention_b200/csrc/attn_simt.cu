@@ -1,5 +1,5 @@
-// Pyramid attention on CUDA cores (fp32 FMA): the path for fp32 inputs and for
-// shapes the tensor-core kernel does not take (64-row query blocks).
+// Pyramid attention on CUDA cores (fp32 FMA): the path for fp32 inputs (the
+// tensor-core kernel takes bf16 with 64- and 128-row query blocks).
 //
 // Method: adaptive pyramid attention (top168.com article on PSA, component
 // three: the probability distribution stays consistent).  Row i of query block

@@ -1,5 +1,8 @@
 // Pyramid attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
-// bf16 inputs, fp32 accumulation, 128-row query blocks, d in {64, 128}.
+// bf16 inputs, fp32 accumulation, 128-row query blocks, d in {64, 128}.  A
+// 64-row query block runs in the same 128-row tiles with rows 64-127 dead (no
+// softmax, no stores): half the tensor work is wasted, against a CUDA-core
+// kernel.
 //
 // Method: adaptive pyramid attention (top168.com article on PSA, component
 // three: one probability distribution over all kept keys) with the paper's
@@ -90,6 +93,7 @@ struct __align__(64) TcParams {
   float* lse;
   int* err;
   int Hq, Hkv, N, Nq, Nk, causal, n_rows;
+  int qb;                                   // query rows per block: 128, or 64 (rows 64-127 dead)
   float scale_log2;
 };
 
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mbar_expect_tx(bar(B_QFULL), C::Q_BYTES);
         for (int h = 0; h < C::HALVES; ++h)
           tma_load_3d(sbase + C::OFF_Q + h * (kBM * 128), &p.tq, bar(B_QFULL), h * 64,
-                      qa * kBM, bhq);
+                      qa * p.qb, bhq);
       }
       ++iq;
       for (int t = 0; t < T; ++t) {
@@ -271,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           int* mpos = reinterpret_cast<int*>(mt_base + 128 + 512);          // [128]
           const bool special = cur.in_tile && (cur.j == p.Nk - 1 ||
                                (p.causal && cur.l == 0 &&
-                                (cur.j + 1) * 64 - 1 >= qa * kBM));
+                                (cur.j + 1) * 64 - 1 >= qa * p.qb));
           const bool slow = __any_sync(0xffffffffu, special);
           if (!slow) {
             if (lane < 16) {
@@ -443,6 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int st = (warp - kSoftWarp0) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
+    const bool dead = r >= p.qb;             // warp-uniform (qb is 64 or 128)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t T_Ss = T_S + st * 128 + lane_off;
     constexpr int HD = D / kStreams;         // merged O columns written by this warpgroup
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (item < 0) continue;
       const int T = row_work(p.counts[item]).tiles;
       const int qa = item % p.Nq, bhq = item / p.Nq;
-      const int qpos = qa * kBM + r;
+      const int qpos = qa * p.qb + r;
       float m = -INFINITY, lsum = 0.f;
       for (int t = st; t < T; t += 2, ++ns) {
         const int gt = g + t, ms = gt % MS;
@@ -465,6 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
              warp_wait(bar(B_MFULL + ms), (gt / MS) & 1, abort_flag, p.err);
         if (!ok) continue;
         tc_fence_after();
+        if (dead) {
+          // rows past a 64-row query block (whole warps): no softmax, no
+          // stores; their P rows are never read into a live row of O
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_MEMPTY + ms));
+          tc_fence_before();
+          mbar_arrive(bar(B_PFULL + st));
+          continue;
+        }
         const unsigned char* mt_base = smem + C::OFF_META + ms * C::META_BYTES;
         const bool slow = *reinterpret_cast<const int*>(mt_base + 64) != 0;
         const float* cb = reinterpret_cast<const float*>(mt_base);            // [16] chunk biases
@@ -609,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         L += ls_[i] * f[i];
       }
       const float inv = keys ? 1.f / L : 0.f;
-      const bool row_ok = qpos < p.N;
+      const bool row_ok = !dead && qpos < p.N;
       __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D + st * HD;
       const bool have_o = T > 0 && __all_sync(0xffffffffu, ok) &&
                           warp_wait(bar(B_OFULL), nb & 1, abort_flag, p.err);
@@ -693,7 +707,8 @@ cudaError_t launch_tc_typed(const TcParams& prm, int rows, cudaStream_t st) {
 }  // namespace
 
 bool attention_tc_supported(const psa_params_t& p) {
-  return p.dtype == PSA_BF16 && p.q_blk == 128 && p.kv_blk == 64 && (p.d == 64 || p.d == 128);
+  return p.dtype == PSA_BF16 && (p.q_blk == 128 || p.q_blk == 64) && p.kv_blk == 64 &&
+         (p.d == 64 || p.d == 128);
 }
 
 cudaError_t launch_attention_tc(const psa_params_t& p, const Layout& L, float scale,
@@ -718,6 +733,7 @@ cudaError_t launch_attention_tc(const psa_params_t& p, const Layout& L, float sc
   prm.Hq = p.Hq; prm.Hkv = p.Hkv; prm.N = p.N; prm.Nq = L.Nq; prm.Nk = L.Nk;
   prm.causal = p.causal;
   prm.n_rows = BHq * L.Nq;
+  prm.qb = p.q_blk;
   prm.scale_log2 = scale * kLog2e;
   return p.d == 128 ? launch_tc_typed<128>(prm, prm.n_rows, st)
                     : launch_tc_typed<64>(prm, prm.n_rows, st);
