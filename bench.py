@@ -72,11 +72,11 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "3fcecd4c344d457b"): 470.370304e6 + 90.855424e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "90ed9b8ad7f847a4"): 474.866432e6 + 91.868416e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
-BWD_TRAFFIC = {("wan2.1_1.3b", 12, "bc04b1e4ab04e483"): 1873.167616e6 + 1333.184256e6}
+BWD_TRAFFIC = {("wan2.1_1.3b", 12, "f48ced556586e6b7"): 1977.520640e6 + 1383.334912e6}
 
 
 def attn_source_hash(sources=ATTN_SOURCES) -> str:
