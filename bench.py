@@ -72,7 +72,7 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "90ed9b8ad7f847a4"): 474.866432e6 + 91.868416e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "e303b466a379d07d"): 472.947712e6 + 91.191296e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
