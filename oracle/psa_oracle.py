@@ -291,9 +291,9 @@ def assign_levels(z: np.ndarray, tau: Sequence[float], N: int, bq: int, bk: int,
     With ``max_level`` (``block_max_levels``), every kept level is then
     lowered to at most its block's max_level (finer, never coarser; pruned
     blocks stay pruned).
-    Readings: the exclusive cumulative mass (so the top block always gets
-    level 0), the quotas as cumulative fractions of the visible blocks rounded
-    up, and the override order are this build's."""
+    Readings where the pages leave the step open: the exclusive cumulative
+    mass (so the top block always gets level 0), the quotas as cumulative
+    fractions of the visible blocks rounded up, and the override order."""
     if rule not in ("threshold", "quantile"):
         raise ValueError(rule)
     Nq, Nk = z.shape
