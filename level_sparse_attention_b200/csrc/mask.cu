@@ -254,7 +254,12 @@ constexpr int kCand = 32 * kCandPerLane;
 constexpr int kCandPerLaneS = 8;
 constexpr int kCandS = 32 * kCandPerLaneS;
 
-__host__ __device__ inline size_t assign_key_bytes(int K, int n2) {
+// Shared-memory bytes of one row's keys.  K > 0: the register path (a
+// candidate set past kCandPerLane keys per lane).  K = 0: all n2 keys (for
+// the bitonic sort of the whole row) and a candidate set.  K < 0, the compact
+// path of long rows: the visible blocks' P as floats and a candidate set.
+__host__ __device__ inline size_t assign_key_bytes(int K, int n2, int Nk) {
+  if (K < 0) return (size_t)((Nk + 31) & ~31) * 4 + (size_t)kCandS * 8;
   return K == 0 ? (size_t)(n2 + kCandS) * 8 : (K > kCandPerLane ? (size_t)kCand * 8 : 0);
 }
 
@@ -321,7 +326,7 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
   const int lev_stride = (a.Nk + 15) & ~15;
   // keys in shared memory: all n2 of them for the shared-memory sort, the
   // candidate set for the register path
-  const size_t key_bytes = assign_key_bytes(K, n2);
+  const size_t key_bytes = assign_key_bytes(K, n2, a.Nk);
   unsigned long long* key = reinterpret_cast<unsigned long long*>(smem) + (size_t)warp * (key_bytes / 8);
   int8_t* lev = reinterpret_cast<int8_t*>(smem + (size_t)rows_per_cta * key_bytes) +
                 (size_t)warp * lev_stride;
@@ -460,6 +465,101 @@ __global__ void assign_kernel(MaskArgs a, int n2, int rows_per_cta, int nrows,
       }
       warp_bitonic_desc<K>(v);
       levels_from_sorted<K>(v, nvis, rule, lev);
+    }
+  } else if constexpr (K < 0) {
+    // Compact path of long rows: P of the visible blocks as floats.  The
+    // candidate cut as below; a row whose cut does not fit ranks every block
+    // against every other (exact; the launch takes this path only when the
+    // cut is expected to fit).
+    float* pv = reinterpret_cast<float*>(key);
+    unsigned long long* cand = key + (((a.Nk + 31) & ~31) >> 1);
+    for (int i = lane; i < nvis; i += 32) pv[i] = expf(z[i] - mx) * inv;
+    __syncwarp();
+    bool done = false;
+    const float target = a.tau[kLevels - 1] + 1e-3f;
+    const int kq = rule.quota[kLevels - 1];
+    if (rule.quantile ? kq <= kCandS : target <= 0.99f) {
+      auto enough = [&](float t, int* cnt) {
+        float m = 0.f;
+        int c = 0;
+        for (int i = lane; i < nvis; i += 32) {
+          const float pi = pv[i];
+          const bool in = pi >= t;
+          m += in ? pi : 0.f;
+          c += in;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          m += __shfl_xor_sync(0xffffffffu, m, o);
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+        }
+        *cnt = c;
+        return rule.quantile ? c >= kq : m >= target;
+      };
+      float pmax = 0.f;
+      for (int i = lane; i < nvis; i += 32) pmax = fmaxf(pmax, pv[i]);
+      pmax = warp_max(pmax);
+      int m_hi, m;
+      float lo = 0.f, hi = pmax, t;
+      if (enough(hi, &m_hi)) {
+        t = hi;
+        m = m_hi;
+      } else {
+        int m_lo = nvis;
+        for (int it = 0; it < 40; ++it) {
+          if (m_lo <= kCandS) break;
+          const float mid = 0.5f * (lo + hi);
+          if (!(mid > lo && mid < hi)) break;
+          int c;
+          if (enough(mid, &c)) {
+            lo = mid;
+            m_lo = c;
+          } else {
+            hi = mid;
+          }
+        }
+        t = lo;
+        m = m_lo;
+      }
+      if (m <= kCandS) {
+        int base = 0;
+        for (int i0 = 0; i0 < nvis; i0 += 32) {
+          const int i = i0 + lane;
+          const float pi = i < nvis ? pv[i] : 0.f;
+          const bool in = i < nvis && pi >= t;
+          const unsigned bal = __ballot_sync(0xffffffffu, in);
+          if (in)
+            cand[base + __popc(bal & ((1u << lane) - 1))] =
+                ((unsigned long long)__float_as_uint(pi) << 32) | (0xffffffffu - (unsigned)i);
+          base += __popc(bal);
+        }
+        __syncwarp();
+        unsigned long long v[kCandPerLaneS];
+#pragma unroll
+        for (int r = 0; r < kCandPerLaneS; ++r) {
+          const int i = lane * kCandPerLaneS + r;
+          v[r] = i < m ? cand[i] : 0ull;
+        }
+        warp_bitonic_desc<kCandPerLaneS>(v);
+        levels_from_sorted<kCandPerLaneS>(v, m, rule, lev);
+        done = true;
+      }
+    }
+    if (!done) {
+      // every block's rank (P descending, ties to the lower index) and the
+      // mass ranked before it, by comparison with every other block
+      for (int j = lane; j < nvis; j += 32) {
+        const float pj = pv[j];
+        float c = 0.f;
+        int rank = 0;
+        for (int i = 0; i < nvis; ++i) {
+          const float pi = pv[i];
+          const bool before = pi > pj || (pi == pj && i < j);
+          c += before ? pi : 0.f;
+          rank += before;
+        }
+        lev[j] = rule.level(c, rank);
+      }
     }
   } else {
     for (int i = lane; i < n2; i += 32) key[i] = make_key(i);
@@ -692,8 +792,15 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
   const MaskArgs a = make_mask_args(p, L, scale);
   const int n2 = next_pow2(L.Nk < 32 ? 32 : L.Nk);
   const bool in_regs = n2 <= 1024;          // register sort; larger rows sort in shared memory
-  const int K = in_regs ? n2 / 32 : 0;
-  const size_t per_row = assign_key_bytes(K, n2) + ((L.Nk + 15) & ~15);
+  // Long rows: the compact path (P as floats, a candidate set), unless the
+  // candidate cut cannot apply (a last threshold within 1% of the whole mass,
+  // or a quantile quota past the candidate set), where every row sorts all
+  // its keys.
+  const int quota3 = (int)ceil((double)p.tau[kLevels - 1] * (double)L.Nk);
+  const bool cut = p.assign == PSA_ASSIGN_QUANTILE ? quota3 <= kCandS
+                                                    : p.tau[kLevels - 1] + 1e-3f <= 0.99f;
+  const int K = in_regs ? n2 / 32 : (cut ? -1 : 0);
+  const size_t per_row = assign_key_bytes(K, n2, L.Nk) + ((L.Nk + 15) & ~15);
   int rows_per_cta = (int)((96 * 1024) / per_row);
   rows_per_cta = rows_per_cta < 1 ? 1 : (rows_per_cta > 2 ? 2 : rows_per_cta);
   const size_t smem = per_row * rows_per_cta;
@@ -714,7 +821,7 @@ cudaError_t launch_assign(const psa_params_t& p, const Layout& L, float scale, c
     case 256: return go(assign_kernel<8>);
     case 512: return go(assign_kernel<16>);
     case 1024: return go(assign_kernel<32>);
-    default: return go(assign_kernel<0>);
+    default: return K < 0 ? go(assign_kernel<-1>) : go(assign_kernel<0>);
   }
 }
 

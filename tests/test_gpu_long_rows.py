@@ -149,3 +149,53 @@ def test_backward_rows_past_the_list_cache(kind):
     _compare_grad(gq, ref.dQ, "dQ")
     _compare_grad(gk, ref.dK, "dK")
     _compare_grad(gv, ref.dV, "dV")
+
+
+def _ramp_inputs(w):
+    """Q and K whose block logits rise by s * a0 = 0.002 per KV block: every
+    query row is a0 * (e_0 + 256 e_1), every key of block j is
+    (j mod 256) e_0 + (j div 256) e_1, so q . k = a0 * j exactly in bf16."""
+    inp = W.make_inputs(w)
+    a0 = 0.002 * np.sqrt(w.d)
+    q = np.zeros((w.B, w.Hq, w.N, w.d), dtype=np.float32)
+    q[..., 0], q[..., 1] = a0, 256.0 * a0
+    j = np.arange(w.N) // w.kv_blk
+    k = np.zeros((w.B, w.Hkv, w.N, w.d), dtype=np.float32)
+    k[..., 0], k[..., 1] = j % 256, j // 256
+    inp.q, inp.k = W.f32_to_bf16_bits(q), W.f32_to_bf16_bits(k)
+    return inp
+
+
+@pytest.mark.parametrize("profile", ["peaked", "flat", "quantile"])
+def test_mask_long_rows_compact_assignment(profile):
+    """The assignment of rows of 1032 blocks, which keeps only P and a
+    candidate set in shared memory, against the oracle's map on sampled rows.
+    peaked: the workload's own inputs and thresholds (the candidate cut holds
+    about a tenth of the row).  flat: block logits rising by 0.002 per block,
+    so neighbouring P differ by 0.2% and tau_3 = 0.98 keeps about 970 blocks,
+    past the candidate set: every block is ranked against every other.
+    quantile: the quantile rule with K_3 = ceil(0.2 * 1032) = 207."""
+    if profile == "quantile":
+        w = W.with_overrides(_workload(128, seed=56), assign="quantile")
+        tau = (0.05, 0.1, 0.15, 0.2)
+        inp = W.make_inputs(w)
+    elif profile == "flat":
+        w = _workload(128, seed=55)
+        tau = (0.3, 0.6, 0.8, 0.98)
+        inp = _ramp_inputs(w)
+    else:
+        w = _workload(128, seed=54)
+        tau = W.thresholds(w)
+        inp = W.make_inputs(w)
+    run = G.run_stages(w, inp, tau=tau)
+    gm = run.level_map.cpu().numpy()[0, 0]
+    Q, K, V = inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0), inp.as_f64("v", 0, 0)
+    pyr = O.build_pyramid(K, V)
+    z = O.block_logits(O.query_block_means(Q, w.q_blk)[SAMPLE], pyr, w.kv_blk, 1.0 / np.sqrt(w.d))
+    mask = O.assign_levels(z, tau, w.N, w.q_blk, w.kv_blk, rule=w.assign)
+    kept = (mask.level_map >= 0).sum(-1)
+    if profile == "flat":
+        assert kept.min() > 900            # well past the 256-block candidate set
+    elif profile == "quantile":
+        assert kept.max() <= 207
+    assert G.map_mismatch_report(gm[SAMPLE], mask, tau, rule=w.assign)[0] == 0
