@@ -72,11 +72,11 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "e303b466a379d07d"): 472.947712e6 + 91.191296e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "4ac2c4cbe2a93a8a"): 469.957888e6 + 90.933760e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")
-BWD_TRAFFIC = {("wan2.1_1.3b", 12, "f48ced556586e6b7"): 1977.520640e6 + 1383.334912e6}
+BWD_TRAFFIC = {("wan2.1_1.3b", 12, "de7109ecc7e51404"): 1945.523200e6 + 1369.462528e6}
 
 
 def attn_source_hash(sources=ATTN_SOURCES) -> str:
