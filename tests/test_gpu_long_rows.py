@@ -151,22 +151,25 @@ def test_backward_rows_past_the_list_cache(kind):
     _compare_grad(gv, ref.dV, "dV")
 
 
-def _ramp_inputs(w):
+def _ramp_inputs(w, pairs=False):
     """Q and K whose block logits rise by s * a0 = 0.002 per KV block: every
     query row is a0 * (e_0 + 256 e_1), every key of block j is
-    (j mod 256) e_0 + (j div 256) e_1, so q . k = a0 * j exactly in bf16."""
+    (j mod 256) e_0 + (j div 256) e_1, so q . k = a0 * j exactly in bf16.
+    With pairs, blocks 2i and 2i + 1 share the keys of 2i: exactly equal P."""
     inp = W.make_inputs(w)
     a0 = 0.002 * np.sqrt(w.d)
     q = np.zeros((w.B, w.Hq, w.N, w.d), dtype=np.float32)
     q[..., 0], q[..., 1] = a0, 256.0 * a0
     j = np.arange(w.N) // w.kv_blk
+    if pairs:
+        j = j & ~1
     k = np.zeros((w.B, w.Hkv, w.N, w.d), dtype=np.float32)
     k[..., 0], k[..., 1] = j % 256, j // 256
     inp.q, inp.k = W.f32_to_bf16_bits(q), W.f32_to_bf16_bits(k)
     return inp
 
 
-@pytest.mark.parametrize("profile", ["peaked", "flat", "quantile"])
+@pytest.mark.parametrize("profile", ["peaked", "flat", "quantile", "ties", "causal"])
 def test_mask_long_rows_compact_assignment(profile):
     """The assignment of rows of 1032 blocks, which keeps only P and a
     candidate set in shared memory, against the oracle's map on sampled rows.
@@ -174,15 +177,23 @@ def test_mask_long_rows_compact_assignment(profile):
     about a tenth of the row).  flat: block logits rising by 0.002 per block,
     so neighbouring P differ by 0.2% and tau_3 = 0.98 keeps about 970 blocks,
     past the candidate set: every block is ranked against every other.
-    quantile: the quantile rule with K_3 = ceil(0.2 * 1032) = 207."""
+    quantile: the quantile rule with K_3 = ceil(0.2 * 1032) = 207.  ties: the
+    flat rise with blocks paired to exactly equal P, through the pairwise
+    ranking (ties to the lower index; no mismatch may hide as a near tie).
+    causal: the causal VLM shape, where a row sees only the blocks up to its
+    diagonal."""
     if profile == "quantile":
         w = W.with_overrides(_workload(128, seed=56), assign="quantile")
         tau = (0.05, 0.1, 0.15, 0.2)
         inp = W.make_inputs(w)
-    elif profile == "flat":
+    elif profile in ("flat", "ties"):
         w = _workload(128, seed=55)
         tau = (0.3, 0.6, 0.8, 0.98)
-        inp = _ramp_inputs(w)
+        inp = _ramp_inputs(w, pairs=profile == "ties")
+    elif profile == "causal":
+        w = _workload(128, causal=True, seed=57)
+        tau = W.thresholds(w)
+        inp = W.make_inputs(w)
     else:
         w = _workload(128, seed=54)
         tau = W.thresholds(w)
@@ -191,11 +202,17 @@ def test_mask_long_rows_compact_assignment(profile):
     gm = run.level_map.cpu().numpy()[0, 0]
     Q, K, V = inp.as_f64("q", 0, 0), inp.as_f64("k", 0, 0), inp.as_f64("v", 0, 0)
     pyr = O.build_pyramid(K, V)
-    z = O.block_logits(O.query_block_means(Q, w.q_blk)[SAMPLE], pyr, w.kv_blk, 1.0 / np.sqrt(w.d))
-    mask = O.assign_levels(z, tau, w.N, w.q_blk, w.kv_blk, rule=w.assign)
+    # causally a row's visible blocks depend on its index: every row is assigned
+    rows = np.arange(w.Nq) if w.causal else np.array(SAMPLE)
+    z = O.block_logits(O.query_block_means(Q, w.q_blk)[rows], pyr, w.kv_blk, 1.0 / np.sqrt(w.d))
+    mask = O.assign_levels(z, tau, w.N, w.q_blk, w.kv_blk, w.causal, w.forced_prefix_tokens,
+                           rule=w.assign)
     kept = (mask.level_map >= 0).sum(-1)
-    if profile == "flat":
+    if profile in ("flat", "ties"):
         assert kept.min() > 900            # well past the 256-block candidate set
     elif profile == "quantile":
         assert kept.max() <= 207
-    assert G.map_mismatch_report(gm[SAMPLE], mask, tau, rule=w.assign)[0] == 0
+    unexplained, _, near_tie = G.map_mismatch_report(gm[rows], mask, tau, rule=w.assign)
+    assert unexplained == 0
+    if profile == "ties":
+        assert near_tie == 0
