@@ -27,9 +27,13 @@ CASES = {
     # grouped queries (2 per KV head), causal, N = 1000
     "bf16_gqa_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=4, Hkv=2, grid=(1, 25, 40),
                                         coarse=(1, 7, 10), seed=13, target="fixed"),
-    # CUDA-core path for bf16 with 64-row query blocks, causal
+    # 64-row query blocks (rows 64-127 of the tensor-core tiles idle), causal
     "bf16_q64_causal": W.with_overrides(BASE["qwen2.5_vl_7b"], Hq=2, Hkv=1, grid=(1, 20, 33),
                                         coarse=(1, 5, 9), seed=14, q_blk=64, target="fixed"),
+    # d = 64 (products of keys 0-63 issued before the rest of the softmax) with 64-row
+    # query blocks, text prefix forced to level 0
+    "bf16_d64_q64": W.with_overrides(BASE["cogvideox_5b"], Hq=2, Hkv=2, grid=(1, 20, 38),
+                                     coarse=(1, 5, 10), seed=18, q_blk=64, target="fixed"),
     # CUDA-core path, fp32, d = 128, 128-row query blocks
     "f32_d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=2, Hkv=2, dtype="f32",
                                  grid=(1, 18, 40), coarse=(1, 5, 10), seed=15, target="fixed"),
