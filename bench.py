@@ -72,7 +72,7 @@ def parse():
 # has changed since the counters were taken has no entry, and the roofline's
 # traffic is then null.
 ATTN_SOURCES = ("attn_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh")
-ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "4ac2c4cbe2a93a8a"): 469.957888e6 + 90.933760e6}
+ATTN_TRAFFIC = {("wan2.1_1.3b", 12, "2cd6a4b28733912d"): 476.693248e6 + 91.385600e6}
 # the same for one launch of the attention-gradient kernel
 BWD_SOURCES = ("attn_bwd_tc.cu", "sm100_ptx.cuh", "psa_internal.cuh", "tile_walk.cuh",
                "bwd_internal.cuh")

@@ -80,8 +80,8 @@ struct Cfg {
   static constexpr int OFF_META = OFF_V + VSTAGES * KV_BYTES;   // per table: bias[128], kpos[128]
   static constexpr int META_BYTES = 128 + 1024;                // chunk biases, flag, per-key tables
   static constexpr int OFF_BAR = OFF_META + MSTAGES * META_BYTES;
-  static constexpr int OFF_XCH = OFF_BAR + 512;                 // stream merge [2][streams][128][2]
-  static constexpr int OFF_LIST = OFF_XCH + 2 * kStreams * 128 * 8;  // the query block's work list
+  static constexpr int OFF_XCH = OFF_BAR + 512;                 // stream 0's (max, sum): [2][128][2]
+  static constexpr int OFF_LIST = OFF_XCH + 2 * 128 * 8;        // the query block's work list
   static constexpr int SMEM = OFF_LIST + 2 * kListCache * 4 + 1024;   // two list copies + slack
 };
 
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   constexpr int B_SFULL = B_MEMPTY + MS, B_PHALF = B_SFULL + kStreams;
   constexpr int B_PFULL = B_PHALF + kStreams;
   constexpr int B_OFULL = B_PFULL + kStreams, B_OFREE = B_OFULL + 1;
-  constexpr int B_FINAL = B_OFREE + 1, NBARS = B_FINAL + 1;
+  constexpr int B_FINAL = B_OFREE + 1, B_XFULL = B_FINAL + 1, NBARS = B_XFULL + 8;
   static_assert(NBARS * 8 + 16 <= 512, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -203,8 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(bar(B_PFULL + i), 128);             // P of all keys written
     }
     mbar_init(bar(B_OFULL), 1);                      // the block's last PV completed
-    mbar_init(bar(B_OFREE), 128 * kStreams);         // both accumulators read out
+    mbar_init(bar(B_OFREE), 128);                    // both accumulators read out (warpgroup 1)
     mbar_init(bar(B_FINAL), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(B_XFULL + i), 32);   // [block parity][quad]: (max, sum) handed over
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -458,18 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // block.  Thread = query row r of the block (TMEM lane r).  The row's
     // scores of a tile are read from S_st twice: pass 1 (all 128 at once)
     // takes the tile maximum, pass 2 the exponentials, 64 keys at a time.  At the end of the block
-    // the two streams' (max, sum) are exchanged through shared memory and a
-    // named barrier (every warp takes it once per block, on every path), and
-    // each warpgroup writes half of the merged O columns.
+    // warpgroup 0 hands its stream's (max, sum) to warpgroup 1, which merges
+    // the two streams and writes O, while warpgroup 0 starts the next block.
     const int st = (warp - kSoftWarp0) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const bool dead = r >= p.qb;             // warp-uniform (qb is 64 or 128)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t T_Ss = T_S + st * 128 + lane_off;
-    constexpr int HD = D / kStreams;         // merged O columns written by this warpgroup
-    constexpr int OC = HD < 32 ? HD : 32;
-    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [2][streams][128][2]
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);   // [block parity][128][max, sum]
     const float sc = p.scale_log2;
     const uint64_t sc2 = f2pack(sc, sc);
     int g = 0, ns = 0, nb = 0;               // tiles before this block, stream tiles, blocks with work
@@ -627,63 +625,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tc_fence_before();
         mbar_arrive(bar(B_PFULL + st));
       }
-      // ---- end of the query block: merge the two streams
-      float* xb = xch + (nb & 1) * (kStreams * 128 * 2);
-      xb[(st * 128 + r) * 2] = m;
-      xb[(st * 128 + r) * 2 + 1] = lsum;
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + quad), "r"(32 * kStreams) : "memory");
-      float ms_[kStreams], ls_[kStreams];
-#pragma unroll
-      for (int i = 0; i < kStreams; ++i) {
-        ms_[i] = xb[(i * 128 + r) * 2];
-        ls_[i] = xb[(i * 128 + r) * 2 + 1];
+      // ---- end of the query block.  Warpgroup 0 hands its (max, sum) to
+      // warpgroup 1 through shared memory and an mbarrier per warp, and goes
+      // on to the next block's first tile; warpgroup 1 merges the two streams
+      // and writes the whole row of O and the LSE.  The buffer and barrier
+      // alternate by block parity: warpgroup 0 reaches the end of block
+      // nb + 2 only after the issuer has seen block nb's accumulators
+      // released, i.e. after warpgroup 1 read block nb's values.
+      const int xid = nb & 1;
+      float* xb = xch + xid * (128 * 2);
+      const uint32_t xbar = bar(B_XFULL + 4 * xid + quad);
+      if (st == 0) {
+        if (T > 0) {
+          xb[r * 2] = m;
+          xb[r * 2 + 1] = lsum;
+          mbar_arrive(xbar);
+          ++nb;
+        }
+        g += T;
+        continue;
       }
-      const float M = fmaxf(ms_[0], ms_[1]);
+      float m0 = -INFINITY, l0 = 0.f;
+      if (T > 0) {
+        ok = ok && warp_wait(xbar, (nb >> 1) & 1, abort_flag, p.err);
+        m0 = xb[r * 2];
+        l0 = xb[r * 2 + 1];
+      }
+      const float M = fmaxf(m0, m);
       const bool keys = M > -INFINITY;                  // the row kept at least one key
-      float f[kStreams], L = 0.f;
-#pragma unroll
-      for (int i = 0; i < kStreams; ++i) {
-        f[i] = ms_[i] > -INFINITY ? ex2(ms_[i] - M) : 0.f;
-        L += ls_[i] * f[i];
-      }
+      const float f0 = m0 > -INFINITY ? ex2(m0 - M) : 0.f;
+      const float f1 = m > -INFINITY ? ex2(m - M) : 0.f;
+      const float L = l0 * f0 + lsum * f1;
       const float inv = keys ? 1.f / L : 0.f;
       const bool row_ok = !dead && qpos < p.N;
-      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D + st * HD;
+      __nv_bfloat16* dst = p.O + ((long long)bhq * p.N + qpos) * D;
       const bool have_o = T > 0 && __all_sync(0xffffffffu, ok) &&
                           warp_wait(bar(B_OFULL), nb & 1, abort_flag, p.err);
       if (have_o) tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += OC) {
-        float o[OC];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
 #pragma unroll
-        for (int i = 0; i < OC; ++i) o[i] = 0.f;
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
         if (have_o) {
 #pragma unroll
           for (int i = 0; i < kStreams; ++i) {
             if (i < T) {                     // stream i holds tiles
-              uint32_t u[OC];
-              tmem_ldn<OC>(T_O + i * D + lane_off + st * HD + c0, u);
+              uint32_t u[32];
+              tmem_ldn<32>(T_O + i * D + lane_off + c0, u);
               tmem_ld_wait();
-              reg_fence<OC>(u);
+              reg_fence<32>(u);
+              const float fi = i == 0 ? f0 : f1;
 #pragma unroll
-              for (int k = 0; k < OC; ++k) o[k] = fmaf(__uint_as_float(u[k]), f[i], o[k]);
+              for (int k = 0; k < 32; ++k) o[k] = fmaf(__uint_as_float(u[k]), fi, o[k]);
             }
           }
         }
         if (row_ok) {
-          uint32_t pk[OC / 2];
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < OC / 2; ++i) {
+          for (int i = 0; i < 16; ++i) {
             __nv_bfloat162 hh = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
             pk[i] = *reinterpret_cast<uint32_t*>(&hh);
           }
           uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-          for (int i = 0; i < OC / 8; ++i)
+          for (int i = 0; i < 4; ++i)
             d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (row_ok && p.lse && st == 0)
+      if (row_ok && p.lse)
         p.lse[(long long)bhq * p.N + qpos] = keys ? (M + log2f(L)) * kLn2 : -INFINITY;
       if (T > 0) {
         // the accumulators may be overwritten by the next block's PVs
