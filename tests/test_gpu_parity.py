@@ -373,3 +373,52 @@ def test_attention_logit_jumps_across_tiles(boost):
     ref_O, ref_lse = O.pyramid_attention(Q, O.build_pyramid(K, V), lm, bq, bk, 1.0 / np.sqrt(d))
     G.compare_out(G.to_f64(out[0, 0]), ref_O, "bf16")
     G.compare_lse(lse[0, 0].cpu().numpy().astype(np.float64), ref_lse, "bf16")
+
+
+SEQUENCE_CASES = {
+    # d = 128, 128-row query blocks; N = 1000 (last query block 104 rows, last KV block 40)
+    "d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=192, Hkv=192, grid=(1, 20, 50),
+                             coarse=(1, 5, 13), seed=31, target="fixed"),
+    # d = 64 (the split PV), N = 986
+    "d64": W.with_overrides(BASE["cogvideox_5b"], Hq=192, Hkv=192, n_text=0, grid=(1, 29, 34),
+                            coarse=(1, 8, 9), forced_prefix_tokens=0, seed=32, target="fixed"),
+    # 64-row query blocks (rows 64-127 of each tile idle), grouped queries
+    "q64_gqa": W.with_overrides(BASE["wan2.1_1.3b"], Hq=96, Hkv=48, grid=(1, 20, 50),
+                                coarse=(1, 5, 13), seed=33, q_blk=64, target="fixed"),
+}
+
+
+def sequence_map(rng, Nq, Nk):
+    """A row keeps no block (a quarter of the rows), or 1 to 16 random blocks
+    at random levels: 0 to 8 packed tiles per query block, mixed along every
+    CTA's sequence of blocks."""
+    m = np.full((Nq, Nk), -1, dtype=np.int8)
+    for a in range(Nq):
+        if rng.random() < 0.25:
+            continue
+        n = int(rng.choice([1, 2, 3, 4, 6, 10, 16]))
+        js = rng.permutation(Nk)[:n]
+        m[a, js] = rng.integers(0, 4, size=len(js))
+    return m
+
+
+@pytest.mark.parametrize("name", sorted(SEQUENCE_CASES))
+def test_attention_block_sequences(name):
+    """Each persistent CTA walks about ten query blocks in a row here, with tile
+    counts from 0 to 8 in random order.  At the end of each block one softmax
+    warpgroup hands its stream's (max, sum) to the other and starts the next
+    block while the other writes O, through buffers and barriers that
+    alternate by block; blocks without keys take no part in the alternation.
+    Every row of every head against the oracle on the same map."""
+    w = SEQUENCE_CASES[name]
+    inp = W.make_inputs(w)
+    rng = np.random.default_rng(zlib.crc32(f"sequences/{name}".encode()))
+    m = np.stack([sequence_map(rng, w.Nq, w.Nk) for _ in range(w.B * w.Hq)])
+    m = m.reshape(w.B, w.Hq, w.Nq, w.Nk)
+    assert w.B * w.Hq * w.Nq >= 8 * 148
+    run = G.run_stages(w, inp, external_map=m)
+    ref = G.oracle_heads(w, inp, [(b, h) for b in range(w.B) for h in range(w.Hq)], level_map=m)
+    gO, glse = G.to_f64(run.O), run.lse.cpu().numpy().astype(np.float64)
+    for (b, h), r in ref.items():
+        G.compare_out(gO[b, h], r.O, w.dtype)
+        G.compare_lse(glse[b, h], r.lse, w.dtype)
