@@ -163,3 +163,17 @@ def compare_lse(gpu_lse: np.ndarray, ref_lse: np.ndarray, dtype: str):
 
 def rand_map(rng, Nq, Nk, lo=-1, hi=4) -> np.ndarray:
     return rng.integers(lo, hi, size=(Nq, Nk)).astype(np.int8)
+
+
+def sequence_map(rng, Nq, Nk) -> np.ndarray:
+    """A row keeps no block (a quarter of the rows), or 1 to 16 random blocks
+    at random levels: 0 to 8 packed tiles per query block, mixed along every
+    persistent CTA's sequence of blocks when there are many query blocks."""
+    m = np.full((Nq, Nk), -1, dtype=np.int8)
+    for a in range(Nq):
+        if rng.random() < 0.25:
+            continue
+        n = int(rng.choice([1, 2, 3, 4, 6, 10, 16]))
+        js = rng.permutation(Nk)[:n]
+        m[a, js] = rng.integers(0, 4, size=len(js))
+    return m

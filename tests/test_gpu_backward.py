@@ -142,6 +142,43 @@ def test_backward_on_external_maps(name, kind):
             assert np.all(gq[:, :, rows] == 0)
 
 
+SEQUENCE_CASES = {
+    # d = 128 and d = 64, 128-row query blocks (the tensor-core kernel); N = 1000 and 986
+    "d128": W.with_overrides(BASE["wan2.1_1.3b"], Hq=192, Hkv=192, grid=(1, 20, 50),
+                             coarse=(1, 5, 13), seed=51, target="fixed"),
+    "d64": W.with_overrides(BASE["cogvideox_5b"], Hq=192, Hkv=192, n_text=0, grid=(1, 29, 34),
+                            coarse=(1, 8, 9), forced_prefix_tokens=0, seed=52, target="fixed"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SEQUENCE_CASES))
+def test_backward_block_sequences(name):
+    """About ten query blocks per persistent CTA, of 0 to 8 tiles in random
+    order (a quarter keep no block): dQ accumulates in TMEM over each block's
+    tiles and is stored at its end, and dK, dV are added row by row into the
+    level accumulators across blocks.  Every head's gradients against the
+    oracle (the criterion of the other cases, over the whole tensors), and
+    exact zeros where nothing is kept."""
+    w = SEQUENCE_CASES[name]
+    inp = W.make_inputs(w)
+    rng = np.random.default_rng(zlib.crc32(f"bwd-sequences/{name}".encode()))
+    m = np.stack([G.sequence_map(rng, w.Nq, w.Nk) for _ in range(w.B * w.Hq)])
+    m = m.reshape(w.B, w.Hq, w.Nq, w.Nk)
+    assert w.B * w.Hq * w.Nq >= 8 * 148
+    run = G.run_stages(w, inp, external_map=m)
+    dO, dO64 = _grad_out(w, zlib.crc32(f"dO-sequences/{name}".encode()))
+    gq, gk, gv = _run_backward(w, inp, run, dO, m)
+    ref = _oracle(w, inp, m, dO64)
+    compare_grad(gq, ref.dQ, w.dtype, "dQ")
+    compare_grad(gk, ref.dK, w.dtype, "dK")
+    compare_grad(gv, ref.dV, w.dtype, "dV")
+    # query blocks that keep nothing pass no gradient: their dQ rows are 0
+    for h in range(w.Hq):
+        for a in np.nonzero((m[0, h] < 0).all(axis=1))[0]:
+            rows = slice(a * w.q_blk, min((a + 1) * w.q_blk, w.N))
+            assert np.all(gq[0, h, rows] == 0)
+
+
 @pytest.mark.parametrize("name", ["bf16_d128", "bf16_gqa_causal", "tiny_f32"])
 def test_backward_after_fused_forward_uses_its_work_list(name):
     """level_map = NULL: the backward walks the list psa_forward left in the

@@ -388,20 +388,6 @@ SEQUENCE_CASES = {
 }
 
 
-def sequence_map(rng, Nq, Nk):
-    """A row keeps no block (a quarter of the rows), or 1 to 16 random blocks
-    at random levels: 0 to 8 packed tiles per query block, mixed along every
-    CTA's sequence of blocks."""
-    m = np.full((Nq, Nk), -1, dtype=np.int8)
-    for a in range(Nq):
-        if rng.random() < 0.25:
-            continue
-        n = int(rng.choice([1, 2, 3, 4, 6, 10, 16]))
-        js = rng.permutation(Nk)[:n]
-        m[a, js] = rng.integers(0, 4, size=len(js))
-    return m
-
-
 @pytest.mark.parametrize("name", sorted(SEQUENCE_CASES))
 def test_attention_block_sequences(name):
     """Each persistent CTA walks about ten query blocks in a row here, with tile
@@ -413,7 +399,7 @@ def test_attention_block_sequences(name):
     w = SEQUENCE_CASES[name]
     inp = W.make_inputs(w)
     rng = np.random.default_rng(zlib.crc32(f"sequences/{name}".encode()))
-    m = np.stack([sequence_map(rng, w.Nq, w.Nk) for _ in range(w.B * w.Hq)])
+    m = np.stack([G.sequence_map(rng, w.Nq, w.Nk) for _ in range(w.B * w.Hq)])
     m = m.reshape(w.B, w.Hq, w.Nq, w.Nk)
     assert w.B * w.Hq * w.Nq >= 8 * 148
     run = G.run_stages(w, inp, external_map=m)
